@@ -1,0 +1,411 @@
+"""Benchmark: the NVFP4 DiT-block linear set at 2048^2 through libnvfp4.
+
+One step = one pass of the whole hot path over one batch of 16896 tokens (16384 image + 512 text),
+hidden 4608:
+    quantise x_qkv (dynamic amax)  -> QKV GEMM [13824 x 4608] + bias + per-head q/k RMSNorm
+    quantise x_attn                -> out-proj GEMM [4608 x 4608] + bias
+    quantise x_ffn                 -> up GEMM [24576 x 4608] + gated SiLU + NVFP4 re-quantisation
+    (up's NVFP4 output)            -> down GEMM [4608 x 12288] + residual + per-channel gate
+Weights are quantised once before timing (they are static).  Every activation is 156 MB, larger
+than the 126 MB L2, so each step streams its inputs from HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+One JSON line on rank 0.  Under torchrun each rank runs an independent replica on its own GPU (the
+path has no exchange step); the time is the max over ranks and the value counts all ranks' work.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from epilogue_gemm_nvfp4_b200 import workloads as W  # noqa: E402
+
+METRIC = "fused NVFP4 linear TFLOPS and % of B200 dense FP4 peak; us per DiT-block linear set"
+UNIT = "TFLOP/s"
+WORKLOAD = "dit_block_linear_set_2048sq"
+NOMINAL_FP4_TFLOPS = 9000.0   # NVIDIA's dense FP4 figure for B200
+BF16_TO_FP4 = 4.0             # nominal dense FP4 / dense bf16 tensor-core rate (9 / 2.25)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"], hbm=d["hbm_gbs"], src="measured")
+    return dict(bf16=1590.0, bf16_sus=1400.0, hbm=6650.0, src="fallback")
+
+
+def layer_flops(M):
+    H, F = W.HIDDEN, W.FFN
+    return dict(qkv=2.0 * M * 3 * H * H, out=2.0 * M * H * H, up=2.0 * M * 2 * F * H, down=2.0 * M * H * F)
+
+
+# ------------------------------------------------------------------------------------------
+# distributed plumbing (replicas)
+# ------------------------------------------------------------------------------------------
+
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, ws: int) -> float:
+    if ws == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        reasons = set()
+        for r in rows:
+            for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                            ("pcap", "sw_power_cap")):
+                if r[k].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["smax"] for r in rows),
+                "power_w_max": max(r["power"] for r in rows), "samples": len(rows), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------------------------------
+# native arm
+# ------------------------------------------------------------------------------------------
+
+class BlockSet:
+    """Device state of the DiT-block linear set: static NVFP4 weights, activations, outputs."""
+
+    def __init__(self, seed=7, M=W.IMG_TOKENS_2K + W.PROMPT_T):
+        from epilogue_gemm_nvfp4_b200 import binding as B
+        self.B = B
+        cases = W.block_2k(seed=seed, M=M)
+        self.M = M
+        self.cases = cases
+        dev = torch.device("cuda")
+        q, o, u, d = cases["qkv"], cases["out"], cases["up"], cases["down"]
+        self.x = {k: cases[k].x.to(dev) for k in ("qkv", "out", "up")}
+        self.wq = {k: B.quantize(cases[k].w.to(dev)) for k in ("qkv", "out", "up", "down")}
+        self.bias = {k: cases[k].bias.to(dev) for k in ("qkv", "out")}
+        ex = q.extras
+        self.qk = dict(gamma_q=ex["gamma_q"].to(dev), gamma_k=ex["gamma_k"].to(dev), eps=ex["eps"],
+                       q_col0=ex["q_col0"], k_col0=ex["k_col0"], qk_cols=ex["qk_cols"], head_dim=ex["head_dim"])
+        self.res = d.extras["residual"].to(dev)
+        self.gate = d.extras["gate"].to(dev)
+        # activation NVFP4 buffers and outputs, allocated once
+        self.aq = {k: B.QTensor.empty(M, W.HIDDEN) for k in ("qkv", "out", "up")}
+        self.up_q = B.QTensor.empty(M, W.FFN)
+        self.out = {"qkv": torch.empty(M, 3 * W.HIDDEN, dtype=torch.bfloat16, device=dev),
+                    "out": torch.empty(M, W.HIDDEN, dtype=torch.bfloat16, device=dev),
+                    "down": torch.empty(M, W.HIDDEN, dtype=torch.bfloat16, device=dev)}
+        # static decode scale of the up projection's NVFP4 output, calibrated once on this input
+        self.up_q.g.fill_(1.0)
+        aq = B.quantize(self.x["up"], out=self.aq["up"])
+        probe = B.linear(aq, self.wq["up"], "gated_silu")
+        torch.cuda.synchronize()
+        self.up_q.g.fill_(float(probe.abs().max().float().item()) / 2688.0)
+        del probe
+        torch.cuda.synchronize()
+
+    def step(self, ev=None):
+        """One pass of the hot path; `ev` (dict of event lists) brackets each op when given."""
+        B = self.B
+
+        def mark(name, i):
+            if ev is not None:
+                ev[name][i].record()
+        mark("quant_qkv", 0); B.quantize(self.x["qkv"], out=self.aq["qkv"]); mark("quant_qkv", 1)
+        mark("qkv", 0)
+        B.linear(self.aq["qkv"], self.wq["qkv"], "qknorm", bias=self.bias["qkv"], out=self.out["qkv"], **self.qk)
+        mark("qkv", 1)
+        mark("quant_out", 0); B.quantize(self.x["out"], out=self.aq["out"]); mark("quant_out", 1)
+        mark("out", 0); B.linear(self.aq["out"], self.wq["out"], "bias", bias=self.bias["out"], out=self.out["out"])
+        mark("out", 1)
+        mark("quant_up", 0); B.quantize(self.x["up"], out=self.aq["up"]); mark("quant_up", 1)
+        mark("up", 0); B.linear(self.aq["up"], self.wq["up"], "gated_silu", out_fp4=self.up_q, want_bf16=False)
+        mark("up", 1)
+        mark("down", 0)
+        B.linear(self.up_q, self.wq["down"], "resid_gate", residual=self.res, gate=self.gate, out=self.out["down"])
+        mark("down", 1)
+
+    LAUNCHES_PER_STEP = 3 * 3 + 4   # per activation: amax, quantise, finalise; four GEMMs
+
+
+OPS = ("quant_qkv", "qkv", "quant_out", "out", "quant_up", "up", "down")
+
+
+def run_native(args, ws, rank, local):
+    from epilogue_gemm_nvfp4_b200 import binding as B
+    B.load()
+    bs = BlockSet()
+    M = bs.M
+    fl = layer_flops(M)
+    step_flops = sum(fl.values())
+
+    for _ in range(args.warmup):
+        bs.step()
+    torch.cuda.synchronize()
+    B.check_device_error()
+
+    # device-timed region: K steps, per-op events on the launching (current) stream
+    ev = {k: [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+              for _ in range(args.steps)] for k in OPS}
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record()
+        for i in range(args.steps):
+            bs.step({k: ev[k][i] for k in OPS})
+        stop.record()
+        torch.cuda.synchronize()
+    barrier(ws)
+    B.check_device_error()
+    ms_local = start.elapsed_time(stop)
+    ms = max_over_ranks(ms_local, ws)
+    per_op = {k: statistics.mean(e[0].elapsed_time(e[1]) for e in ev[k]) for k in OPS}
+    ms_step = ms / args.steps
+    value = step_flops * ws / (ms_step * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers: H2D of the step's activations and residual
+    # from pinned memory, the step, D2H of its outputs, all inside the timed region
+    host_in = {k: bs.x[k].cpu().pin_memory() for k in ("qkv", "out", "up")}
+    host_res = bs.res.cpu().pin_memory()
+    host_out = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in bs.out.items()}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values()) + host_res.numel() * host_res.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        for k in host_in:
+            bs.x[k].copy_(host_in[k], non_blocking=True)
+        bs.res.copy_(host_res, non_blocking=True)
+        bs.step()
+        for k in host_out:
+            host_out[k].copy_(bs.out[k], non_blocking=True)
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    t2.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(s2.elapsed_time(t2), ws) / e2e_steps
+    barrier(ws)
+
+    pk = peaks()
+    dominant = max(("qkv", "out", "up", "down"), key=lambda k: fl[k])
+    achieved = fl[dominant] / (per_op[dominant] * 1e-3) / 1e12
+    peak_fp4 = pk["bf16_sus"] * BF16_TO_FP4
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4 e2m1 x e4m3/16 -> fp32 acc", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens": M, "hidden": W.HIDDEN, "ffn": W.FFN, "heads": W.N_HEADS,
+                   "head_dim": W.HEAD_DIM, "seed": 7, "parallelism": f"replicas x{ws}",
+                   "l2": "inputs larger than L2 (each activation 156 MB)"},
+        "us_per_block_linear_set": round(ms_step * 1e3, 1),
+        "frac_of_nominal_fp4": round(value / ws / NOMINAL_FP4_TFLOPS, 4),
+        "per_op_us": {k: round(v * 1e3, 1) for k, v in per_op.items()},
+        "per_gemm_tflops": {k: round(fl[k] / (per_op[k] * 1e-3) / 1e12, 1) for k in ("qkv", "out", "up", "down")},
+        "roofline": {"bound": "tensor", "kernel": f"nvfp4_gemm_kernel ({dominant}: gated SiLU + requant)",
+                     "achieved": round(achieved, 1), "peak": round(peak_fp4, 1), "unit": "TFLOP/s",
+                     "frac": round(achieved / peak_fp4, 4),
+                     "peak_note": f"{pk['src']} sustained bf16 {pk['bf16_sus']} x {BF16_TO_FP4} (nominal FP4/bf16)",
+                     "frac_of_nominal_9pf": round(achieved / NOMINAL_FP4_TFLOPS, 4),
+                     "traffic": None},
+        "quantize_roofline": None,
+        "e2e": {"value": round(step_flops * ws / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": BlockSet.LAUNCHES_PER_STEP * args.steps,
+    }
+    qbytes = 2.5625 * M * W.HIDDEN
+    qus = per_op["quant_qkv"] * 1e3
+    out["quantize_roofline"] = {"bound": "hbm", "kernel": "amax + quantize_kernel (x [16896, 4608])",
+                                "achieved": round(qbytes / (qus * 1e-6) / 1e9, 1), "peak": pk["hbm"], "unit": "GB/s",
+                                "frac": round(qbytes / (qus * 1e-6) / 1e9 / pk["hbm"], 4),
+                                "note": "algorithmic bytes 2.5625 B/elem (amax pass reads another 2 B/elem, "
+                                        "not counted)"}
+    out["clocks"] = clk.summary()
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+    return out
+
+
+# ------------------------------------------------------------------------------------------
+# the oracle on the host cores (cpu_baseline leg and the reference arm)
+# ------------------------------------------------------------------------------------------
+
+class OracleSample:
+    """A bounded sample of the block workload for the oracle: `rows` tokens; every layer keeps whole
+    heads / gate pairs and the full reduction width.  Weights are quantised once (static, untimed)."""
+
+    def __init__(self, rows=64, seed=7):
+        from oracle import nvfp4_oracle as O
+        self.O = O
+        rng = np.random.default_rng(seed)
+        H, F, K = W.HIDDEN, W.FFN, W.HIDDEN
+        f = lambda a: W.to_bf16(a).float().numpy()
+        self.rows, self.rng, self.f = rows, rng, f
+        w = {"qkv": f(W.normal(rng, (1536, K), 0.015)), "out": f(W.normal(rng, (512, K), 0.015)),
+             "up": f(W.normal(rng, (1024, K), 0.015)), "down": f(W.normal(rng, (512, F), 0.01))}
+        self.wq = {k: O.quantize(v) for k, v in w.items()}
+        self.bias = {"qkv": f(W.normal(rng, (1536,), 0.01)), "out": f(W.normal(rng, (512,), 0.01))}
+        self.gam = f(W.uniform(rng, (256,), 0.5, 1.5))
+        self.gate = W.uniform(rng, (512,), 0.0, 1.0)
+        self.flops = 2.0 * rows * K * (1536 + 512 + 1024) + 2.0 * rows * F * 512
+        self.note = (f"{rows} tokens x (QKV 1536 + out 512 + up 1024 + down 512 weight rows), full K; "
+                     "activation quantisation, GEMMs, epilogues and requant timed; weight quantisation not")
+
+    def step(self):
+        """Draw one batch of activations, then time the oracle's pass over it.  Returns seconds."""
+        O, f, rng, rows = self.O, self.f, self.rng, self.rows
+        x = {k: f(W.normal(rng, (rows, W.HIDDEN))) for k in ("qkv", "out", "up")}
+        x_dn = f(W.normal(rng, (rows, W.FFN)))
+        res = f(W.normal(rng, (rows, 512)))
+        t0 = time.perf_counter()
+        O.linear(O.quantize(x["qkv"]), self.wq["qkv"], "qknorm", bias=self.bias["qkv"], gamma_q=self.gam,
+                 gamma_k=self.gam, eps=1e-6, q_col0=0, k_col0=512, qk_cols=512)
+        O.linear(O.quantize(x["out"]), self.wq["out"], "bias", bias=self.bias["out"])
+        O.linear(O.quantize(x["up"]), self.wq["up"], "gated_silu", out_g=np.float32(0.01))
+        O.linear(O.quantize(x_dn), self.wq["down"], "resid_gate", residual=res, gate=self.gate)
+        return time.perf_counter() - t0
+
+
+def cpu_baseline(seconds=15.0):
+    smp = OracleSample()
+    dt = 0.0
+    reps = 0
+    while reps < 2 or dt < seconds:
+        dt += smp.step()
+        reps += 1
+    return {"value": round(smp.flops * reps / dt / 1e12, 6), "unit": UNIT, "cores": torch.get_num_threads(),
+            "kind": "oracle", "sample": f"{reps} x [{smp.note}]", "seconds": round(dt, 2)}
+
+
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return None
+    smp = OracleSample()
+    note = smp.note
+    times = [smp.step() for _ in range(args.warmup + args.steps)][args.warmup:]
+    ms = statistics.mean(times) * 1e3
+    val = smp.flops / (ms * 1e-3) / 1e12
+    return {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle; fp32 quantiser steps)",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "tokens": W.IMG_TOKENS_2K + W.PROMPT_T, "hidden": W.HIDDEN,
+                       "sample": note},
+            "cpu_baseline": {"value": round(val, 6), "unit": UNIT, "cores": torch.get_num_threads(),
+                             "kind": "oracle", "sample": note},
+            "e2e": {"value": round(val, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("native", "reference"), default="native")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        res = run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    ws, rank, local = dist_init()
+    res = run_native(args, ws, rank, local)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

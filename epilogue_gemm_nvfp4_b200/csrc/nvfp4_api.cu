@@ -1,0 +1,331 @@
+// Host side of libnvfp4: argument checks, TMA descriptors, tile configuration and launches.
+// The library allocates no memory; the only device state it owns is one sticky error word per
+// device, a module-scope __device__ variable.
+#include <cudaTypedefs.h>
+
+#include <cstdlib>
+#include <mutex>
+
+#include "../../include/nvfp4.h"
+#include "gemm.cuh"
+#include "ptx.cuh"
+#include "quantize.cuh"
+
+using namespace nvfp4;
+
+namespace {
+
+__device__ unsigned int g_device_error;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  int sm_count = 0;
+  unsigned int* error_word = nullptr;
+  bool smem_attr_set[2][4] = {};
+};
+
+std::mutex g_mutex;
+DeviceState g_devices[kMaxDevices];
+
+// Per-device set-up, done once with that device current: SM count and the address of the error word.
+nvfp4_status device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState& st = g_devices[dev];
+  if (!st.ready) {
+    if (cudaDeviceGetAttribute(&st.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&st.error_word), g_device_error) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    st.ready = true;
+  }
+  *out = &st;
+  return NVFP4_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+uint64_t wait_timeout_ns() {
+  static uint64_t ns = [] {
+    const char* e = std::getenv("NVFP4_WAIT_TIMEOUT_MS");
+    long ms = e ? std::strtol(e, nullptr, 10) : 1000;
+    if (ms <= 0) ms = 1000;
+    return static_cast<uint64_t>(ms) * 1000000ull;
+  }();
+  return ns;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+int64_t k_atoms_of(int64_t cols) { return (cols / 16 + 3) / 4; }
+
+int64_t ld_codes_of(const nvfp4_tensor* t) { return t->ld_codes ? t->ld_codes : t->cols / 2; }
+
+// Checks shared by every NVFP4 tensor argument.
+nvfp4_status check_tensor(const nvfp4_tensor* t, bool need_scale) {
+  if (!t || !t->codes || !t->scales || (need_scale && !t->tensor_scale)) return NVFP4_ERR_INVALID_ARG;
+  if (t->rows < 0 || t->cols <= 0) return NVFP4_ERR_INVALID_ARG;
+  if (t->cols % 16) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  const int64_t ld = ld_codes_of(t);
+  if (ld < t->cols / 2) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(t->codes) || (ld % 16) || !aligned16(t->scales) || (t->tensor_scale && !aligned4(t->tensor_scale)))
+    return NVFP4_ERR_MISALIGNED;
+  return NVFP4_OK;
+}
+
+nvfp4_status launch_status() { return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+int elementwise_grid(int64_t work_items, int items_per_cta, int sm_count) {
+  int64_t g = (work_items + items_per_cta - 1) / items_per_cta;
+  const int64_t cap = static_cast<int64_t>(sm_count) * 8;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return static_cast<int>(g);
+}
+
+// 2-D TMA descriptor over packed E2M1 codes viewed as bytes: [rows][cols/2], box 128 x 128 bytes,
+// 128-byte swizzle (the layout the tensor-core descriptors expect).
+nvfp4_status make_code_map(CUtensorMap* map, const nvfp4_tensor* t) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return NVFP4_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(t->cols / 2), static_cast<cuuint64_t>(t->rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_codes_of(t))};
+  cuuint32_t box[2] = {128, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, t->codes, dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+int tile_n_for(int64_t N, int64_t K, int32_t kind) {
+  if (K < 64 || K % 64) return 0;
+  if (kind == NVFP4_EPI_QKNORM || kind == NVFP4_EPI_GATED_SILU) return (N > 0 && N % 256 == 0) ? 256 : 0;
+  if (kind == NVFP4_EPI_BIAS || kind == NVFP4_EPI_RESID_GATE) {
+    if (N > 0 && N % 256 == 0) return 256;
+    if (N > 0 && N % 128 == 0) return 128;
+  }
+  return 0;
+}
+
+template <int BN, int KIND>
+nvfp4_status launch_gemm(DeviceState* st, const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& args,
+                         cudaStream_t stream) {
+  using C = GemmCfg<BN>;
+  auto kernel = nvfp4_gemm_kernel<BN, KIND>;
+  bool& attr = st->smem_attr_set[BN == 256 ? 1 : 0][KIND];
+  if (!attr) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    attr = true;
+  }
+  const int grid = args.num_tiles < st->sm_count ? args.num_tiles : st->sm_count;
+  kernel<<<grid, 256, C::SMEM_BYTES, stream>>>(ma, mb, args);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t nvfp4_version(void) { return 100; }
+
+const char* nvfp4_status_string(nvfp4_status s) {
+  switch (s) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case NVFP4_ERR_MISALIGNED: return "misaligned pointer or leading dimension";
+    case NVFP4_ERR_CUDA: return "CUDA runtime error";
+    case NVFP4_ERR_DEVICE_TIMEOUT: return "device-side pipeline wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t nvfp4_scale_bytes(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols <= 0) return 0;
+  const int64_t r = (rows + 127) / 128 * 128;
+  return static_cast<size_t>(r * k_atoms_of(cols) * 4);
+}
+
+int64_t nvfp4_scale_offset(int64_t r, int64_t kb, int64_t cols) { return scale_offset(r, kb, k_atoms_of(cols)); }
+
+int32_t nvfp4_linear_tile_n(int64_t N, int64_t K, int32_t kind) { return tile_n_for(N, K, kind); }
+
+nvfp4_status nvfp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ldx, float* amax, nvfp4_stream_t stream) {
+  if (!x || !amax || rows < 0 || cols <= 0 || ldx < cols) return NVFP4_ERR_INVALID_ARG;
+  if (cols % 8) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || (ldx * 2) % 16 || !aligned4(amax)) return NVFP4_ERR_MISALIGNED;
+  DeviceState* st;
+  if (nvfp4_status e = device_state(&st)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(amax, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (rows == 0) return NVFP4_OK;
+  const int grid = elementwise_grid(rows * cols / 8, 256 * 4, st->sm_count);
+  amax_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), rows, cols, ldx,
+                                   reinterpret_cast<unsigned int*>(amax));
+  return launch_status();
+}
+
+nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int32_t compute_scale,
+                            const nvfp4_tensor* out, nvfp4_stream_t stream) {
+  if (!x || !out || rows < 0 || cols <= 0 || ldx < cols) return NVFP4_ERR_INVALID_ARG;
+  if (nvfp4_status e = check_tensor(out, true)) return e;
+  if (out->rows != rows || out->cols != cols) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(x) || (ldx * 2) % 16) return NVFP4_ERR_MISALIGNED;
+  DeviceState* st;
+  if (nvfp4_status e = device_state(&st)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  auto* codes = static_cast<uint8_t*>(out->codes);
+  auto* scales = static_cast<uint8_t*>(out->scales);
+  const int64_t ld = ld_codes_of(out), ka = k_atoms_of(cols);
+  const int64_t tasks = rows * ((cols + 255) / 256) + 1;
+  const int qgrid = elementwise_grid(tasks, 8 * kQuantUnroll, st->sm_count);
+  if (compute_scale) {
+    if (cudaMemsetAsync(out->tensor_scale, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (rows > 0) {
+      const int agrid = elementwise_grid(rows * cols / 8, 256 * 4, st->sm_count);
+      amax_kernel<<<agrid, 256, 0, s>>>(xb, rows, cols, ldx, reinterpret_cast<unsigned int*>(out->tensor_scale));
+    }
+    quantize_kernel<true><<<qgrid, 256, 0, s>>>(xb, rows, cols, ldx, out->tensor_scale, codes, ld, scales, ka);
+    finalize_scale_kernel<<<1, 1, 0, s>>>(out->tensor_scale);
+  } else {
+    quantize_kernel<false><<<qgrid, 256, 0, s>>>(xb, rows, cols, ldx, out->tensor_scale, codes, ld, scales, ka);
+  }
+  return launch_status();
+}
+
+nvfp4_status nvfp4_dequantize(const nvfp4_tensor* t, void* out_bf16, int64_t ld_out, nvfp4_stream_t stream) {
+  if (!out_bf16) return NVFP4_ERR_INVALID_ARG;
+  if (nvfp4_status e = check_tensor(t, true)) return e;
+  if (ld_out < t->cols) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(out_bf16) || (ld_out * 2) % 16) return NVFP4_ERR_MISALIGNED;
+  if (t->rows == 0) return NVFP4_OK;
+  DeviceState* st;
+  if (nvfp4_status e = device_state(&st)) return e;
+  const int grid = elementwise_grid(t->rows * (t->cols / 16), 256, st->sm_count);
+  dequantize_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(t->codes), ld_codes_of(t), static_cast<const uint8_t*>(t->scales), t->tensor_scale,
+      t->rows, t->cols, k_atoms_of(t->cols), static_cast<__nv_bfloat16*>(out_bf16), ld_out);
+  return launch_status();
+}
+
+nvfp4_status nvfp4_linear(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvfp4_epilogue_desc* epi,
+                          void* out_bf16, int64_t ld_out, const nvfp4_tensor* out_fp4, nvfp4_stream_t stream) {
+  if (!epi) return NVFP4_ERR_INVALID_ARG;
+  if (nvfp4_status e = check_tensor(a, true)) return e;
+  if (nvfp4_status e = check_tensor(w, true)) return e;
+  const int64_t M = a->rows, N = w->rows, K = a->cols;
+  if (w->cols != K) return NVFP4_ERR_INVALID_ARG;
+  if (epi->kind < NVFP4_EPI_BIAS || epi->kind > NVFP4_EPI_RESID_GATE) return NVFP4_ERR_INVALID_ARG;
+  const int BN = tile_n_for(N, K, epi->kind);
+  if (BN == 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30) || K > (int64_t(1) << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  const int64_t n_out = epi->kind == NVFP4_EPI_GATED_SILU ? N / 2 : N;
+  if (epi->bias && !aligned16(epi->bias)) return NVFP4_ERR_MISALIGNED;
+  if (epi->kind == NVFP4_EPI_QKNORM) {
+    if (!epi->gamma_q || !epi->gamma_k || epi->head_dim != 256 || !(epi->eps > 0.0f)) return NVFP4_ERR_INVALID_ARG;
+    if (epi->q_col0 % 256 || epi->k_col0 % 256 || epi->qk_cols % 256 || epi->q_col0 < 0 || epi->k_col0 < 0 ||
+        epi->qk_cols < 0 || epi->q_col0 + epi->qk_cols > N || epi->k_col0 + epi->qk_cols > N)
+      return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(epi->gamma_q) || !aligned16(epi->gamma_k)) return NVFP4_ERR_MISALIGNED;
+  }
+  if (epi->kind == NVFP4_EPI_RESID_GATE) {
+    if (!epi->residual || !epi->gate || epi->ld_residual < n_out) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(epi->residual) || (epi->ld_residual * 2) % 16 || !aligned16(epi->gate)) return NVFP4_ERR_MISALIGNED;
+  }
+  if (epi->out_nvfp4) {
+    if (nvfp4_status e = check_tensor(out_fp4, true)) return e;
+    if (out_fp4->rows != M || out_fp4->cols != n_out) return NVFP4_ERR_INVALID_ARG;
+  } else if (!out_bf16) {
+    return NVFP4_ERR_INVALID_ARG;
+  }
+  if (out_bf16) {
+    if (ld_out < n_out) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(out_bf16) || (ld_out * 2) % 16) return NVFP4_ERR_MISALIGNED;
+  }
+  if (M == 0) return NVFP4_OK;
+  DeviceState* st;
+  if (nvfp4_status e = device_state(&st)) return e;
+
+  CUtensorMap ma, mb;
+  if (nvfp4_status e = make_code_map(&ma, a)) return e;
+  if (nvfp4_status e = make_code_map(&mb, w)) return e;
+
+  GemmArgs g{};
+  g.M = static_cast<int32_t>(M);
+  g.N = static_cast<int32_t>(N);
+  g.K = static_cast<int32_t>(K);
+  g.num_m_blocks = static_cast<int32_t>((M + 127) / 128);
+  g.num_n_blocks = static_cast<int32_t>(epi->kind == NVFP4_EPI_GATED_SILU ? (N / 2) / 128 : N / BN);
+  g.num_tiles = g.num_m_blocks * g.num_n_blocks;
+  g.k_steps = static_cast<int32_t>(K / 64);
+  g.k_atoms = static_cast<int32_t>(k_atoms_of(K));
+  g.sfa = static_cast<const uint8_t*>(a->scales);
+  g.sfb = static_cast<const uint8_t*>(w->scales);
+  g.ga = a->tensor_scale;
+  g.gb = w->tensor_scale;
+  g.bias = static_cast<const __nv_bfloat16*>(epi->bias);
+  g.gamma_q = static_cast<const __nv_bfloat16*>(epi->gamma_q);
+  g.gamma_k = static_cast<const __nv_bfloat16*>(epi->gamma_k);
+  g.eps = epi->eps;
+  g.q_col0 = static_cast<int32_t>(epi->q_col0);
+  g.k_col0 = static_cast<int32_t>(epi->k_col0);
+  g.qk_cols = static_cast<int32_t>(epi->qk_cols);
+  g.residual = static_cast<const __nv_bfloat16*>(epi->residual);
+  g.ld_res = epi->ld_residual;
+  g.gate = epi->gate;
+  g.out = static_cast<__nv_bfloat16*>(out_bf16);
+  g.ld_out = ld_out;
+  if (epi->out_nvfp4) {
+    g.q_codes = static_cast<uint8_t*>(out_fp4->codes);
+    g.ld_q_codes = ld_codes_of(out_fp4);
+    g.q_scales = static_cast<uint8_t*>(out_fp4->scales);
+    g.q_g = out_fp4->tensor_scale;
+    g.q_k_atoms = static_cast<int32_t>(k_atoms_of(n_out));
+  }
+  g.error_word = st->error_word;
+  g.timeout_ns = wait_timeout_ns();
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (epi->kind) {
+    case NVFP4_EPI_BIAS:
+      return BN == 256 ? launch_gemm<256, kEpiBias>(st, ma, mb, g, s) : launch_gemm<128, kEpiBias>(st, ma, mb, g, s);
+    case NVFP4_EPI_RESID_GATE:
+      return BN == 256 ? launch_gemm<256, kEpiResidGate>(st, ma, mb, g, s)
+                       : launch_gemm<128, kEpiResidGate>(st, ma, mb, g, s);
+    case NVFP4_EPI_QKNORM: return launch_gemm<256, kEpiQkNorm>(st, ma, mb, g, s);
+    case NVFP4_EPI_GATED_SILU: return launch_gemm<256, kEpiGatedSilu>(st, ma, mb, g, s);
+  }
+  return NVFP4_ERR_INVALID_ARG;
+}
+
+nvfp4_status nvfp4_get_device_error(nvfp4_stream_t stream) {
+  DeviceState* st;
+  if (nvfp4_status e = device_state(&st)) return e;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (v) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return NVFP4_ERR_CUDA;
+  }
+  return v == 0 ? NVFP4_OK : (v == kErrTimeout ? NVFP4_ERR_DEVICE_TIMEOUT : NVFP4_ERR_CUDA);
+}
+
+}  // extern "C"

@@ -1,0 +1,212 @@
+// Bandwidth-bound NVFP4 kernels: the amax pass, the quantiser, its one-thread finalise step, and the
+// dequantiser.  All loads and stores are 16-byte vectors; a warp covers 256 consecutive elements of
+// a row (16 blocks of 16) per step, so every load and every code store is coalesced.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+constexpr float kTensorScaleDivisor = 2688.0f;  // 6 (largest E2M1) * 448 (largest E4M3)
+
+// Byte offset of the scale of row r, block c in the padded tensor-core layout (k_atoms = blocks per
+// row / 4, rounded up): 512-byte atoms of 128 rows x 4 blocks, K-major atom order.
+__host__ __device__ __forceinline__ int64_t scale_offset(int64_t r, int64_t c, int64_t k_atoms) {
+  return ((r >> 7) * k_atoms + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
+}
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_absmax_bits(uint32_t w) {
+  return max(w & 0x7FFFu, (w >> 16) & 0x7FFFu);
+}
+
+// ------------------------------------------------------------------------------------------
+// amax: max |x| over a bf16 matrix.  For finite bf16, |x| orders like its 15-bit magnitude field,
+// so the reduction runs on integers and one atomicMax per CTA publishes the fp32 bit pattern.
+// ------------------------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(256) amax_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
+                                                   int64_t cols, int64_t ldx, unsigned int* __restrict__ out_bits) {
+  uint32_t m = 0;
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (ldx == cols) {
+    const int64_t groups = rows * cols / 8;  // 8 bf16 per 16-byte load
+    const uint4* p = reinterpret_cast<const uint4*>(x);
+    int64_t g = tid;
+    for (; g + 3 * nthreads < groups; g += 4 * nthreads) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = ld_stream(p + g + u * nthreads);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        m = max(m, max(max(bf16x2_absmax_bits(v[u].x), bf16x2_absmax_bits(v[u].y)),
+                       max(bf16x2_absmax_bits(v[u].z), bf16x2_absmax_bits(v[u].w))));
+    }
+    for (; g < groups; g += nthreads) {
+      const uint4 v = ld_stream(p + g);
+      m = max(m, max(max(bf16x2_absmax_bits(v.x), bf16x2_absmax_bits(v.y)),
+                     max(bf16x2_absmax_bits(v.z), bf16x2_absmax_bits(v.w))));
+    }
+  } else {
+    const int64_t gpr = cols / 8;
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+      const uint4* p = reinterpret_cast<const uint4*>(x + r * ldx);
+      for (int64_t g = threadIdx.x; g < gpr; g += blockDim.x) {
+        const uint4 v = ld_stream(p + g);
+        m = max(m, max(max(bf16x2_absmax_bits(v.x), bf16x2_absmax_bits(v.y)),
+                       max(bf16x2_absmax_bits(v.z), bf16x2_absmax_bits(v.w))));
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __shared__ uint32_t red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) m = max(m, red[w]);
+    if (m) atomicMax(out_bits, m << 16);  // bf16 magnitude -> fp32 bit pattern
+  }
+}
+
+// g = amax / 2688 (or 1 for an all-zero tensor), in place: the slot held amax bits.
+__global__ void finalize_scale_kernel(float* __restrict__ slot) {
+  const float amax = *slot;
+  *slot = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, kTensorScaleDivisor);
+}
+
+__device__ __forceinline__ float tensor_scale_from(const float* src, bool from_amax) {
+  const float v = *src;
+  if (!from_amax) return v;
+  return (v == 0.0f) ? 1.0f : __fdiv_rn(v, kTensorScaleDivisor);
+}
+
+// The block rule for one 16-element block, given its amax and the tensor decode scale g:
+// returns the E4M3 byte and the fp32 reciprocal of d = e4m3(s) * g (0 when d == 0).
+__device__ __forceinline__ uint32_t block_scale(float amax_b, float g, float& inv) {
+  const float r = __fdiv_rn(amax_b, g);
+  const float sf = __fdiv_rn(r, 6.0f);
+  const uint32_t s = e4m3_satfinite(sf);
+  const float d = __fmul_rn(e4m3_to_float(s), g);
+  inv = (d == 0.0f) ? 0.0f : __frcp_rn(d);
+  return s;
+}
+
+// ------------------------------------------------------------------------------------------
+// quantise.  Warp task = (row, 256-element span).  Lane l holds elements [8l, 8l+8) of the span;
+// lanes 2j and 2j+1 form block j and meet with one shuffle for the block amax.
+// ------------------------------------------------------------------------------------------
+
+constexpr int kQuantUnroll = 4;
+
+template <bool kFromAmax>
+__global__ void __launch_bounds__(256) quantize_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
+                                                       int64_t cols, int64_t ldx, const float* __restrict__ scale_src,
+                                                       uint8_t* __restrict__ codes, int64_t ld_codes,
+                                                       uint8_t* __restrict__ scales, int64_t k_atoms) {
+  const float g = tensor_scale_from(scale_src, kFromAmax);
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t gwarp = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t spans = (cols + 255) / 256;
+  const int64_t total = rows * spans;
+  const int64_t blocks_per_row = cols / 16;
+
+  for (int64_t t0 = gwarp; t0 < total; t0 += nwarps * kQuantUnroll) {
+    uint4 v[kQuantUnroll];
+    int64_t row[kQuantUnroll], col[kQuantUnroll];
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      const int64_t t = t0 + u * nwarps;
+      row[u] = t / spans;
+      col[u] = (t - row[u] * spans) * 256 + lane * 8;
+      v[u] = make_uint4(0, 0, 0, 0);
+      if (t < total && col[u] < cols) v[u] = ld_stream(x + row[u] * ldx + col[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      const int64_t t = t0 + u * nwarps;
+      if (t >= total) break;  // warp-uniform
+      const bool valid = col[u] < cols;
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      float f[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
+      uint32_t mb = max(max(bf16x2_absmax_bits(w[0]), bf16x2_absmax_bits(w[1])),
+                        max(bf16x2_absmax_bits(w[2]), bf16x2_absmax_bits(w[3])));
+      mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 1));
+      const float amax_b = __uint_as_float(mb << 16);
+      float inv;
+      uint32_t s = block_scale(amax_b, g, inv);
+      float q[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(f[i], inv);
+      uint32_t packed = e2m1x8(q);
+      if (inv == 0.0f) packed = 0;
+      if (!valid) s = 0;
+      if (valid) *reinterpret_cast<uint32_t*>(codes + row[u] * ld_codes + col[u] / 2) = packed;
+      // four consecutive blocks' scales share one aligned 32-bit word of the scale layout
+      const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, s, 2);
+      const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, s, 4);
+      const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, s, 6);
+      const int64_t blk = col[u] / 16;
+      if ((lane & 7) == 0 && blk < blocks_per_row) {
+        *reinterpret_cast<uint32_t*>(scales + scale_offset(row[u], blk, k_atoms)) =
+            s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      }
+    }
+  }
+
+  // zero the scale rows that pad the tensor to a multiple of 128 rows
+  const int64_t pad_rows = ((rows + 127) & ~int64_t(127)) - rows;
+  const int64_t pad_words = pad_rows * k_atoms;
+  const int64_t nthr = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < pad_words; i += nthr) {
+    const int64_t r = rows + i / k_atoms, a = i % k_atoms;
+    *reinterpret_cast<uint32_t*>(scales + scale_offset(r, a * 4, k_atoms)) = 0u;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// dequantise: one thread per 16-element block.
+// ------------------------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restrict__ codes, int64_t ld_codes,
+                                                         const uint8_t* __restrict__ scales,
+                                                         const float* __restrict__ gptr, int64_t rows, int64_t cols,
+                                                         int64_t k_atoms, __nv_bfloat16* __restrict__ out,
+                                                         int64_t ld_out) {
+  const float g = *gptr;
+  const int64_t bpr = cols / 16;
+  const int64_t total = rows * bpr;
+  const int64_t nthr = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += nthr) {
+    const int64_t r = i / bpr, b = i - r * bpr;
+    const uint2 c = *reinterpret_cast<const uint2*>(codes + r * ld_codes + b * 8);
+    const float d = __fmul_rn(e4m3_to_float(scales[scale_offset(r, b, k_atoms)]), g);
+    uint32_t o[8];
+#pragma unroll
+    for (int i2 = 0; i2 < 8; ++i2) {
+      const uint32_t byte = ((i2 < 4 ? c.x : c.y) >> (8 * (i2 & 3))) & 0xFFu;
+      const __nv_bfloat16 lo = __float2bfloat16_rn(__fmul_rn(e2m1_to_float(byte & 0xFu), d));
+      const __nv_bfloat16 hi = __float2bfloat16_rn(__fmul_rn(e2m1_to_float(byte >> 4), d));
+      o[i2] = static_cast<uint32_t>(__bfloat16_as_ushort(lo)) | (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out + r * ld_out + b * 16);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+}  // namespace nvfp4

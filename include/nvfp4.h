@@ -1,0 +1,176 @@
+/*
+ * nvfp4.h - C ABI of libnvfp4: the NVFP4 quantised linear layer of a flow-matching diffusion
+ * transformer, with the small op that follows each product fused into the GEMM epilogue.
+ *
+ * What is computed comes from "Serving sub-second Ideogram v4 without quality loss" (fal, via
+ * tldrocket.com): the DiT's matrix products run in NVFP4, the 4-bit floating-point format that
+ * Blackwell tensor cores execute natively, and the RMSNorm over 256-wide attention heads or the
+ * gated SiLU that follows a product runs inside the same kernel instead of after a round trip of
+ * the product through memory.  The text-conditioning projection (53248 -> 4608 with a bias) and
+ * the rule that a linear must treat its rows independently come from "Faster Ideogram 4 with Less
+ * Prompt Compute" (sections "Most of the Tensor Was Zero" and "The NF4 Exactness Problem").
+ *
+ * Encoding (the pages do not spell it out; this is the reading the library implements):
+ *   - element: E2M1 code in 4 bits, sign in bit 3, magnitudes {0,.5,1,1.5,2,3,4,6};
+ *   - block:   one unsigned E4M3 scale byte per 16 consecutive elements of a row;
+ *   - tensor:  one fp32 decode scale g; value = e2m1(code) * e4m3(scale) * g.
+ *   Quantisation of a block: r = amax_b / g; s = E4M3(r / 6); d = s * g; code_i = E2M1(x_i * (1/d)),
+ *   each step one binary32 operation rounded to nearest even, E4M3 and E2M1 rounding to nearest even
+ *   and saturating (448, 6).  A block with d == 0 gets codes 0.  The tensor scale computed by
+ *   nvfp4_quantize is g = amax / 2688 (2688 = 6 * 448), or 1 when the tensor is all zero.
+ *
+ * Conventions for every entry point:
+ *   - All pointers inside the structs and all data pointers are DEVICE pointers, owned by the caller.
+ *     The library allocates nothing and frees nothing.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default stream).  Host-side
+ *     argument checks run before anything is launched; when one fails nothing is launched and the
+ *     status says why.  Nothing throws, prints or traps.
+ *   - NVFP4_ERR_CUDA means a CUDA runtime call failed (the launch, or the device has no sm_100a).
+ *   - Device-side failures (a pipeline wait that ran out of time) are recorded in a sticky per-device
+ *     word and reported by nvfp4_get_device_error().
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* nvfp4_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,       /* NULL where a pointer is required, negative size, bad enum      */
+  NVFP4_ERR_UNSUPPORTED_SHAPE = 2, /* a size rule below is not met                                   */
+  NVFP4_ERR_MISALIGNED = 3,        /* a pointer or leading dimension is not 16-byte aligned           */
+  NVFP4_ERR_CUDA = 4,              /* a CUDA runtime call failed                                      */
+  NVFP4_ERR_DEVICE_TIMEOUT = 5     /* a kernel's pipeline wait ran out of time and the kernel gave up */
+} nvfp4_status;
+
+/*
+ * An NVFP4 tensor of `rows` x `cols` logical elements (cols = the reduction dimension K for GEMM
+ * operands).
+ *   codes:        uint8, row r starts at codes + r * ld_codes; element k of the row is the low nibble
+ *                 of byte k/2 when k is even, the high nibble when k is odd.  ld_codes >= cols/2 and a
+ *                 multiple of 16 (0 means cols/2).
+ *   scales:       uint8 E4M3 block scales in the tensor-core scale layout, nvfp4_scale_bytes(rows, cols)
+ *                 bytes: 512-byte atoms of 128 rows x 4 blocks, atoms ordered along K first, then along
+ *                 rows; inside an atom row r, block c is at (r%32)*16 + ((r/32)%4)*4 + c%4 (see
+ *                 nvfp4_scale_offset).  Rows are padded to a multiple of 128 and blocks per row to a
+ *                 multiple of 4; nvfp4_quantize writes 0 into the padding.
+ *   tensor_scale: one fp32, the decode scale g.
+ */
+typedef struct {
+  void* codes;
+  void* scales;
+  float* tensor_scale;
+  int64_t rows;
+  int64_t cols;
+  int64_t ld_codes;
+} nvfp4_tensor;
+
+typedef enum {
+  NVFP4_EPI_BIAS = 0,       /* y = acc + bias                                                      */
+  NVFP4_EPI_QKNORM = 1,     /* y = acc + bias; RMSNorm of every 256-wide head in the q and k ranges */
+  NVFP4_EPI_GATED_SILU = 2, /* y = acc + bias; out = silu(y[:, :N/2]) * y[:, N/2:]                  */
+  NVFP4_EPI_RESID_GATE = 3  /* out = residual + gate[n] * (acc + bias)                              */
+} nvfp4_epilogue_kind;
+
+/*
+ * The op fused after the product acc[m,n] = sum_k a[m,k] * w[n,k] (dequantised operands, fp32
+ * accumulation).  N is w->rows.  The output has N columns, or N/2 for NVFP4_EPI_GATED_SILU.
+ *   bias:          bf16 [N] or NULL (no bias).  Added before any norm or activation.
+ *   QKNORM:        gamma_q, gamma_k bf16 [head_dim]; head_dim must be 256; eps > 0.  Columns
+ *                  [q_col0, q_col0 + qk_cols) are normalised per head with gamma_q, columns
+ *                  [k_col0, k_col0 + qk_cols) with gamma_k: y_h / sqrt(mean(y_h^2) + eps) * gamma.
+ *                  q_col0, k_col0 and qk_cols are multiples of 256; other columns get bias only.
+ *   GATED_SILU:    rows [0, N/2) of w give a, rows [N/2, N) give b; out = a / (1 + exp(-a)) * b.
+ *   RESID_GATE:    residual bf16 [M, ld_residual] (row stride in elements), gate fp32 [N].
+ *   out_nvfp4:     1 = also re-quantise the bf16-rounded output to NVFP4 into `out_fp4` with the
+ *                  caller's static decode scale already stored in out_fp4->tensor_scale (the rule of
+ *                  nvfp4_quantize, so the codes equal nvfp4_quantize of the bf16 output bit for bit).
+ */
+typedef struct {
+  int32_t kind;
+  const void* bias;
+  const void* gamma_q;
+  const void* gamma_k;
+  float eps;
+  int32_t head_dim;
+  int64_t q_col0;
+  int64_t k_col0;
+  int64_t qk_cols;
+  const void* residual;
+  int64_t ld_residual;
+  const float* gate;
+  int32_t out_nvfp4;
+} nvfp4_epilogue_desc;
+
+/*
+ * Quantise a bf16 matrix x [rows, cols] (row stride ldx elements) to NVFP4 into `out`
+ * (out->rows == rows, out->cols == cols).
+ *   compute_scale = 1: compute g = amax(|x|) / 2688 on the device and store it in *out->tensor_scale
+ *                      (an amax pass, the quantise pass and a one-thread finalise, stream-ordered).
+ *   compute_scale = 0: use the g already stored in *out->tensor_scale (a calibrated static scale).
+ * Rules: cols % 16 == 0; x and ldx*2 16-byte aligned; codes and ld_codes 16-byte aligned; scales
+ * 16-byte aligned.  rows == 0 is a no-op.
+ */
+NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int32_t compute_scale,
+                            const nvfp4_tensor* out, nvfp4_stream_t stream);
+
+/*
+ * The fused NVFP4 linear: out = epilogue(a x w^T) on one GPU.
+ *   a:        NVFP4 [M, K] activation.  w: NVFP4 [N, K] weight (nn.Linear layout).
+ *   out_bf16: bf16 [M, ld_out] (row stride in elements) or NULL when only out_fp4 is wanted.
+ *   out_fp4:  NVFP4 [M, n_out] when epi->out_nvfp4 == 1, else ignored (may be NULL).
+ * Rules: K % 64 == 0, K >= 64; N % 128 == 0 (N % 256 == 0 for QKNORM and GATED_SILU); M >= 1 (any);
+ * all pointers and ld_out * 2 16-byte aligned.  The per-row arithmetic does not depend on M: row m of
+ * the output is bitwise the same whatever rows accompany it.
+ */
+NVFP4_API nvfp4_status nvfp4_linear(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvfp4_epilogue_desc* epi,
+                          void* out_bf16, int64_t ld_out, const nvfp4_tensor* out_fp4, nvfp4_stream_t stream);
+
+/* Dequantise t to bf16 [t->rows, ld_out]: value = e2m1(code) * (e4m3(scale) * g), each product in fp32
+ * rounded to nearest even, then rounded to bf16.  Rules as for nvfp4_quantize. */
+NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor* t, void* out_bf16, int64_t ld_out, nvfp4_stream_t stream);
+
+/* max |x| over a bf16 matrix into *amax (device fp32), overwriting it.  The first pass of
+ * nvfp4_quantize(compute_scale = 1), exported so it can be timed and used on its own. */
+NVFP4_API nvfp4_status nvfp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ldx, float* amax,
+                        nvfp4_stream_t stream);
+
+/* Size in bytes of the padded block-scale buffer of a rows x cols NVFP4 tensor. */
+NVFP4_API size_t nvfp4_scale_bytes(int64_t rows, int64_t cols);
+
+/* Byte offset of the scale of row r, 16-element block kb, in a tensor with `cols` columns
+ * (host helper). */
+NVFP4_API int64_t nvfp4_scale_offset(int64_t r, int64_t kb, int64_t cols);
+
+/* Wait for `stream`, then return and clear the sticky device-side error of the current device
+ * (NVFP4_OK when none). */
+NVFP4_API nvfp4_status nvfp4_get_device_error(nvfp4_stream_t stream);
+
+/* Column tile width the GEMM uses for a weight of N rows and K columns and an epilogue kind; it
+ * depends on (N, K, kind) only, never on M.  0 when the shape is unsupported. */
+NVFP4_API int32_t nvfp4_linear_tile_n(int64_t N, int64_t K, int32_t kind);
+
+/* Static string naming a status code. */
+NVFP4_API const char* nvfp4_status_string(nvfp4_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+NVFP4_API int32_t nvfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

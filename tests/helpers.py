@@ -1,0 +1,69 @@
+"""Shared helpers for the parity tests: moving seeded inputs to the GPU and to the oracle."""
+import numpy as np
+import torch
+
+from oracle import nvfp4_oracle as O
+
+
+def f32(t: torch.Tensor) -> np.ndarray:
+    """bf16/fp32 torch tensor (any device) -> float32 numpy (exact for bf16)."""
+    return t.detach().float().cpu().numpy()
+
+
+def oracle_quantize(x_bf16: torch.Tensor, g=None):
+    """Oracle quantisation of a bf16 tensor: (codes [M,K], scales [M,K/16], g)."""
+    return O.quantize(f32(x_bf16), g)
+
+
+def gpu_qtensor_bytes(q):
+    """(packed codes numpy [M,K/2], scale buffer numpy, g float32) of a binding.QTensor."""
+    torch.cuda.synchronize()
+    return q.codes.cpu().numpy(), q.scales.cpu().numpy(), np.float32(q.g.cpu().item())
+
+
+def assert_quant_bitexact(q, ref, M, K):
+    """GPU NVFP4 tensor == oracle (codes, scales, g) byte for byte, padding included."""
+    codes, scales, g = gpu_qtensor_bytes(q)
+    rc, rs, rg = ref
+    assert g == rg, (g, rg)
+    want_codes = O.pack_codes(rc)
+    bad = np.argwhere(codes != want_codes)
+    assert bad.size == 0, f"{len(bad)} code bytes differ, first at {bad[:5].tolist()}"
+    want_scales = O.scales_to_mma_layout(rs)
+    assert scales.shape == want_scales.shape, (scales.shape, want_scales.shape)
+    bad = np.flatnonzero(scales != want_scales)
+    assert bad.size == 0, f"{bad.size} scale bytes differ, first offsets {bad[:5].tolist()}"
+
+
+def normwise_rel_err(got, ref) -> float:
+    return O.rel_err_normwise(got, ref)
+
+
+def elementwise_ok(got, ref, rel=2e-2, floor_frac=1e-2):
+    """Elementwise |got-ref| <= rel * max(|ref|, floor_frac * rms(ref)); returns the worst ratio."""
+    ref = np.asarray(ref, np.float64)
+    got = np.asarray(got, np.float64)
+    rms = np.sqrt(np.mean(ref * ref)) if ref.size else 1.0
+    den = np.maximum(np.abs(ref), floor_frac * rms)
+    return float(np.max(np.abs(got - ref) / den)) / rel
+
+
+def assert_requant_close(q, ref, M, K, max_frac=1e-3):
+    """A fused re-quantised output against the oracle's re-quantisation of its own bf16 output.
+
+    The two bf16 outputs may differ in the last bit, which can move a block scale by one E4M3 step
+    or a code by one E2M1 step.  Everything else must match: the fraction of differing scale bytes
+    and codes stays below ``max_frac`` and every difference is one step.
+    """
+    codes, scales, g = gpu_qtensor_bytes(q)
+    rc, rs, rg = ref
+    assert g == rg
+    got_s = O.scales_from_mma_layout(scales, M, K).astype(np.int64)
+    ds = np.abs(got_s - rs.astype(np.int64))
+    assert ds.max(initial=0) <= 1 and np.mean(ds > 0) <= max_frac, (ds.max(initial=0), np.mean(ds > 0))
+    got_c = O.unpack_codes(codes).astype(np.int64)
+    same_scale = np.repeat(ds == 0, 16, axis=1)
+    mag = lambda c: np.where(c & 8, -(c & 7), c & 7)          # signed magnitude index
+    dc = np.abs(mag(got_c) - mag(rc.astype(np.int64)))
+    dc = np.where(same_scale, dc, 0)
+    assert dc.max(initial=0) <= 1 and np.mean(dc > 0) <= max_frac, (dc.max(initial=0), np.mean(dc > 0))

@@ -1,0 +1,98 @@
+"""The C-ABI library: it loads, exports every function include/nvfp4.h declares, and its host-side
+logic (scale layout helpers, tile choice, argument checks) behaves as documented.  No GPU needed:
+every call here returns before the first CUDA call."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from epilogue_gemm_nvfp4_b200 import binding as B
+from oracle import nvfp4_oracle as O
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "nvfp4.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"NVFP4_API\s+[\w\s\*]+?\b(nvfp4_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(B.EXPORTS)
+
+
+def test_library_loads_and_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.nvfp4_version() >= 100
+    assert B.status_string(B.ERR_MISALIGNED).startswith("misaligned")
+
+
+def test_scale_helpers_match_the_layout_definition(lib):
+    for rows, cols in [(1, 16), (127, 64), (128, 512), (300, 208), (4608, 4608)]:
+        assert lib.nvfp4_scale_bytes(rows, cols) == O.scale_buffer_bytes(rows, cols)
+    rng = np.random.default_rng(0)
+    for _ in range(200):
+        rows, cols = int(rng.integers(1, 2000)), int(rng.integers(1, 400)) * 16
+        r, kb = int(rng.integers(0, rows)), int(rng.integers(0, cols // 16))
+        assert lib.nvfp4_scale_offset(r, kb, cols) == O.scale_atom_offset(r, kb, cols)
+
+
+def test_tile_choice_depends_on_n_k_kind_only(lib):
+    assert B.tile_n(13824, 4608, "qknorm") == 256
+    assert B.tile_n(24576, 4608, "gated_silu") == 256
+    assert B.tile_n(4608, 53248, "bias") in (128, 256)
+    assert B.tile_n(384, 512, "bias") == 128
+    assert B.tile_n(384, 512, "qknorm") == 0          # heads need 256-column tiles
+    assert B.tile_n(512, 96, "bias") == 0             # K % 64
+    assert B.tile_n(200, 512, "bias") == 0            # N % 128
+
+
+def _tensor(rows, cols, ptr=0x10000):
+    return B.CTensor(ptr, ptr, ptr, rows, cols, cols // 2)
+
+
+def test_argument_checks_return_before_any_launch(lib):
+    desc = B.CEpilogue()
+    a, w = _tensor(256, 512), _tensor(512, 512)
+    lin = lambda a_, w_, d_, out=0x10000, ld=512, q=None: lib.nvfp4_linear(
+        ctypes.byref(a_), ctypes.byref(w_), ctypes.byref(d_), out, ld, q, None)
+    assert lib.nvfp4_linear(None, ctypes.byref(w), ctypes.byref(desc), 0x10000, 512, None, None) == B.ERR_INVALID_ARG
+    assert lin(_tensor(256, 512), _tensor(512, 256), desc) == B.ERR_INVALID_ARG          # K mismatch
+    assert lin(_tensor(256, 96), _tensor(512, 96), desc) == B.ERR_UNSUPPORTED_SHAPE      # K % 64
+    assert lin(_tensor(256, 512), _tensor(200, 512), desc) == B.ERR_UNSUPPORTED_SHAPE    # N % 128
+    assert lin(_tensor(256, 512, 0x10008), w, desc) == B.ERR_MISALIGNED
+    assert lin(a, w, desc, out=0x10002) == B.ERR_MISALIGNED
+    assert lin(a, w, desc, ld=100) == B.ERR_INVALID_ARG                                    # ld_out < N
+    assert lin(a, w, desc, out=0) == B.ERR_INVALID_ARG                                     # no output at all
+    bad = B.CEpilogue(kind=7)
+    assert lin(a, w, bad) == B.ERR_INVALID_ARG
+    qk = B.CEpilogue(kind=B.EPI_QKNORM, gamma_q=0x10000, gamma_k=0x10000, eps=1e-6, head_dim=128)
+    assert lin(a, w, qk) == B.ERR_INVALID_ARG                                              # head_dim != 256
+    qk = B.CEpilogue(kind=B.EPI_QKNORM, gamma_q=0x10000, gamma_k=0x10000, eps=1e-6, head_dim=256,
+                     q_col0=0, k_col0=256, qk_cols=512)
+    assert lin(a, w, qk) == B.ERR_UNSUPPORTED_SHAPE                                        # k range past N
+    rg = B.CEpilogue(kind=B.EPI_RESID_GATE)
+    assert lin(a, w, rg) == B.ERR_INVALID_ARG                                              # no residual/gate
+    q = _tensor(256, 256)
+    gs = B.CEpilogue(kind=B.EPI_GATED_SILU, out_nvfp4=1)
+    assert lin(a, w, gs, q=ctypes.byref(_tensor(256, 512))) == B.ERR_INVALID_ARG           # out_fp4 not [M, N/2]
+    # quantise / dequantise / amax
+    t = _tensor(4, 512)
+    assert lib.nvfp4_quantize(None, 4, 512, 512, 1, ctypes.byref(t), None) == B.ERR_INVALID_ARG
+    assert lib.nvfp4_quantize(0x10000, 4, 520, 520, 1, ctypes.byref(_tensor(4, 520)), None) == B.ERR_UNSUPPORTED_SHAPE
+    assert lib.nvfp4_quantize(0x10000, 4, 512, 500, 1, ctypes.byref(t), None) == B.ERR_INVALID_ARG
+    assert lib.nvfp4_quantize(0x10000, 4, 512, 516, 1, ctypes.byref(t), None) == B.ERR_MISALIGNED
+    assert lib.nvfp4_quantize(0x10000, 5, 512, 512, 1, ctypes.byref(t), None) == B.ERR_INVALID_ARG
+    assert lib.nvfp4_dequantize(ctypes.byref(t), None, 512, None) == B.ERR_INVALID_ARG
+    assert lib.nvfp4_amax(0x10000, 4, 512, 512, None, None) == B.ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_a_device_reports_cuda_error(lib):
+    a, w = _tensor(256, 512), _tensor(512, 512)
+    desc = B.CEpilogue()
+    assert lib.nvfp4_linear(ctypes.byref(a), ctypes.byref(w), ctypes.byref(desc), 0x10000, 512, None, None) \
+        == B.ERR_CUDA

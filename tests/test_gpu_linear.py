@@ -1,0 +1,222 @@
+"""GPU parity of the fused NVFP4 linear (nvfp4_linear through the C ABI) against the oracle.
+
+The oracle runs on its own quantisation of the same seeded bf16 inputs; the GPU quantiser is checked
+bit-exact against that quantisation first, so both sides multiply the same NVFP4 operands.  The bar
+for GEMM + epilogue outputs is a normwise max relative error of 2e-2 (bf16 output).  Row independence
+is checked bitwise on the GPU.
+"""
+import numpy as np
+import pytest
+import torch
+
+from epilogue_gemm_nvfp4_b200 import binding as B
+from epilogue_gemm_nvfp4_b200 import workloads as W
+from oracle import nvfp4_oracle as O
+from tests.helpers import (assert_quant_bitexact, assert_requant_close, elementwise_ok, f32, normwise_rel_err,
+                           oracle_quantize)
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+
+
+def gpu_epi_kwargs(case):
+    ex = case.extras
+    if case.epilogue == "qknorm":
+        return dict(gamma_q=ex["gamma_q"].cuda(), gamma_k=ex["gamma_k"].cuda(), eps=ex["eps"], q_col0=ex["q_col0"],
+                    k_col0=ex["k_col0"], qk_cols=ex["qk_cols"], head_dim=ex["head_dim"])
+    if case.epilogue == "resid_gate":
+        return dict(residual=ex["residual"].cuda(), gate=ex["gate"].cuda())
+    return {}
+
+
+def oracle_epi_kwargs(case):
+    ex = case.extras
+    if case.epilogue == "qknorm":
+        return dict(gamma_q=f32(ex["gamma_q"]), gamma_k=f32(ex["gamma_k"]), eps=ex["eps"], q_col0=ex["q_col0"],
+                    k_col0=ex["k_col0"], qk_cols=ex["qk_cols"], head_dim=ex["head_dim"])
+    if case.epilogue == "resid_gate":
+        return dict(residual=f32(ex["residual"]), gate=f32(ex["gate"]))
+    return {}
+
+
+def run_gpu(case, aq=None, out_fp4=None, want_bf16=True):
+    aq = B.quantize(case.x.cuda()) if aq is None else aq
+    wq = B.quantize(case.w.cuda())
+    bias = case.bias.cuda() if case.bias is not None else None
+    out = B.linear(aq, wq, case.epilogue, bias=bias, out_fp4=out_fp4, want_bf16=want_bf16, **gpu_epi_kwargs(case))
+    B.check_device_error()
+    return aq, wq, out
+
+
+def run_oracle(case, rows=None, a_ref=None, w_ref=None, out_g=None):
+    a_ref = oracle_quantize(case.x) if a_ref is None else a_ref
+    w_ref = oracle_quantize(case.w) if w_ref is None else w_ref
+    bias = f32(case.bias) if case.bias is not None else None
+    return a_ref, w_ref, O.linear(a_ref, w_ref, case.epilogue, bias=bias, rows=rows, out_g=out_g,
+                                  **oracle_epi_kwargs(case))
+
+
+def check(got, ref, what):
+    err = normwise_rel_err(got, ref)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    assert err <= TOL, f"{what}: normwise rel err {err:.3e} > {TOL}"
+    return err
+
+
+# ------------------------------------------------------------------------------------------
+# small and ragged cases, whole outputs
+# ------------------------------------------------------------------------------------------
+
+def test_tiny_workload_full(lib):
+    case = W.tiny()
+    aq, wq, out = run_gpu(case)
+    a_ref, w_ref, ref = run_oracle(case)
+    assert_quant_bitexact(aq, a_ref, case.M, case.K)
+    assert_quant_bitexact(wq, w_ref, case.N, case.K)
+    check(f32(out), ref["y"], "tiny")
+    assert elementwise_ok(f32(out), ref["y"]) <= 1.0
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 64), (127, 384, 320), (129, 256, 512), (300, 512, 1024),
+                                   (64, 128, 4608), (257, 768, 192)])
+def test_bias_ragged(lib, M, N, K):
+    case = W.case_bias(M, N, K, seed=M + N + K, w_std=0.05)
+    aq, wq, out = run_gpu(case)
+    _, _, ref = run_oracle(case)
+    check(f32(out), ref["y"], f"bias {M}x{N}x{K}")
+
+
+def test_no_bias(lib):
+    case = W.case_bias(200, 256, 256, seed=3)
+    case.bias = None
+    _, _, out = run_gpu(case)
+    _, _, ref = run_oracle(case)
+    check(f32(out), ref["y"], "no bias")
+
+
+@pytest.mark.parametrize("M", [200, 1])
+def test_qknorm_small(lib, M):
+    case = W.case_qkv(M, n_heads=2, K=512, seed=5)
+    _, _, out = run_gpu(case)
+    _, _, ref = run_oracle(case)
+    check(f32(out), ref["y"], "qknorm")
+    # the normalised heads have rms ~ |gamma| scale, the v range keeps bias-only values
+    got = f32(out)[:, :512].reshape(M, 2, 256)
+    assert np.all(np.sqrt(np.mean(got ** 2, axis=2)) < 2.0)
+
+
+def test_resid_gate_small(lib):
+    case = W.case_ffn_down(150, N=384, F=512, seed=6)
+    _, _, out = run_gpu(case)
+    _, _, ref = run_oracle(case)
+    check(f32(out), ref["y"], "resid_gate")
+
+
+def test_gated_silu_with_requant_small(lib):
+    case = W.case_ffn_up(130, K=512, F=256, seed=7)
+    case.bias = W.to_bf16(np.random.default_rng(70).standard_normal(512).astype(np.float32) * 0.01)
+    a_ref, w_ref, ref = run_oracle(case)
+    g_out = np.float32(np.max(np.abs(ref["bf16"])) / np.float32(2688.0))
+    q = B.QTensor.empty(case.M, case.n_out)
+    q.g.fill_(float(g_out))
+    aq, wq, out = run_gpu(case, out_fp4=q)
+    check(f32(out), ref["y"], "gated silu")
+    # the fused re-quantisation equals the quantiser applied to the kernel's own bf16 output
+    q2 = B.quantize(out, g=float(g_out))
+    torch.cuda.synchronize()
+    assert torch.equal(q.codes, q2.codes)
+    assert torch.equal(q.scales, q2.scales)
+    # and it matches the oracle's re-quantisation of its own bf16 output up to one-step differences
+    assert_requant_close(q, O.quantize(ref["bf16"], g_out), case.M, case.n_out)
+    # fp4-only output (no bf16 written) gives the same codes
+    q3 = B.QTensor.empty(case.M, case.n_out)
+    q3.g.fill_(float(g_out))
+    run_gpu(case, aq=aq, out_fp4=q3, want_bf16=False)
+    assert torch.equal(q.codes, q3.codes) and torch.equal(q.scales, q3.scales)
+
+
+def test_tile_n_128_path_and_k_tail(lib):
+    # N = 384 forces 128-wide tiles (two TMEM accumulators); K = 320 leaves a one-MMA tail stage
+    case = W.case_bias(515, 384, 320, seed=9, w_std=0.05)
+    assert B.tile_n(384, 320, "bias") == 128
+    _, _, out = run_gpu(case)
+    _, _, ref = run_oracle(case)
+    check(f32(out), ref["y"], "bn128")
+
+
+# ------------------------------------------------------------------------------------------
+# row independence (bitwise, on the GPU)
+# ------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T", [512, 1941])
+def test_row_independence_text_projection(lib, T):
+    """The T text rows project identically with or without the 4096 zero image rows appended, and
+    each zero row projects to exactly the bias ("Most of the Tensor Was Zero")."""
+    base = W.text_proj(T)
+    padded = W.text_proj(T, zero_rows=W.IMG_TOKENS_1K)
+    assert torch.equal(padded.x[:T], base.x)
+    wq = B.quantize(base.w.cuda())
+    bias = base.bias.cuda()
+    a1 = B.quantize(base.x.cuda())
+    a2 = B.quantize(padded.x.cuda())
+    assert a1.g.item() == a2.g.item()
+    o1 = B.linear(a1, wq, "bias", bias=bias)
+    o2 = B.linear(a2, wq, "bias", bias=bias)
+    B.check_device_error()
+    assert torch.equal(o1, o2[:T])
+    assert torch.equal(o2[T:], bias.expand(W.IMG_TOKENS_1K, -1))
+
+
+# ------------------------------------------------------------------------------------------
+# full-size workloads: every GPU output against the oracle on sampled rows
+# ------------------------------------------------------------------------------------------
+
+def sample_rows(M, n=48, seed=0):
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, 127, 128, 255, M // 2, M - 129, M - 128, M - 1]
+    rows = np.unique(np.concatenate([[r for r in fixed if 0 <= r < M], rng.choice(M, n, replace=False)]))
+    return rows
+
+
+def test_qkv_1k_sampled(lib):
+    case = W.qkv_1k()
+    aq, wq, out = run_gpu(case)
+    rows = sample_rows(case.M)
+    a_ref = oracle_quantize(case.x)
+    w_ref = oracle_quantize(case.w)
+    assert_quant_bitexact(aq, a_ref, case.M, case.K)
+    _, _, ref = run_oracle(case, rows=rows, a_ref=a_ref, w_ref=w_ref)
+    check(f32(out)[rows], ref["y"], "qkv 1024^2")
+
+
+def test_ffn_1k_chain_sampled(lib):
+    up, down = W.ffn_1k()
+    rows = sample_rows(up.M, n=32, seed=1)
+    a_ref = oracle_quantize(up.x)
+    w_up = oracle_quantize(up.w)
+    _, _, r_up = run_oracle(up, rows=rows, a_ref=a_ref, w_ref=w_up)
+    g_out = np.float32(np.max(np.abs(r_up["bf16"])) / np.float32(2688.0))
+    q = B.QTensor.empty(up.M, up.n_out)
+    q.g.fill_(float(g_out))
+    _, _, out_up = run_gpu(up, out_fp4=q)
+    check(f32(out_up)[rows], r_up["y"], "ffn up")
+    # down projection consumes each side's own fused NVFP4 output
+    res = f32(down.extras["residual"])[rows]
+    gate = f32(down.extras["gate"])
+    oq = O.quantize(r_up["bf16"], g_out)
+    w_dn = oracle_quantize(down.w)
+    r_dn = O.linear(oq, w_dn, "resid_gate", residual=res, gate=gate)
+    wq_dn = B.quantize(down.w.cuda())
+    out_dn = B.linear(q, wq_dn, "resid_gate", residual=down.extras["residual"].cuda(), gate=down.extras["gate"].cuda())
+    B.check_device_error()
+    check(f32(out_dn)[rows], r_dn["y"], "ffn down")
+
+
+@pytest.mark.parametrize("T", [512, 1941])
+def test_text_projection_sampled(lib, T):
+    case = W.text_proj(T)
+    aq, wq, out = run_gpu(case)
+    rows = np.arange(T) if T == 512 else sample_rows(T, n=40, seed=2)
+    _, _, ref = run_oracle(case, rows=rows)
+    check(f32(out)[rows], ref["y"], f"text T={T}")

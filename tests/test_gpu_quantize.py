@@ -1,0 +1,91 @@
+"""GPU parity of the bandwidth kernels through the C ABI: quantise (both scale modes), amax and
+dequantise must equal the oracle byte for byte, padding included."""
+import numpy as np
+import pytest
+import torch
+
+from epilogue_gemm_nvfp4_b200 import binding as B
+from epilogue_gemm_nvfp4_b200 import workloads as W
+from oracle import nvfp4_oracle as O
+from tests.helpers import assert_quant_bitexact, f32, oracle_quantize
+
+pytestmark = pytest.mark.gpu
+
+
+def rand_bf16(rows, cols, seed, scale=1.0, dist="normal"):
+    rng = np.random.default_rng(seed)
+    a = W.student_t(rng, (rows, cols)) if dist == "t" else W.normal(rng, (rows, cols), scale)
+    return W.to_bf16(a)
+
+
+@pytest.mark.parametrize("rows,cols,seed", [(1, 16, 0), (5, 48, 1), (130, 208, 2), (127, 64, 3), (129, 512, 4),
+                                            (300, 4608, 5), (33, 53248, 6)])
+def test_quantize_bitexact_ragged(lib, rows, cols, seed):
+    x = rand_bf16(rows, cols, seed, dist="t" if seed % 2 else "normal")
+    q = B.quantize(x.cuda())
+    assert_quant_bitexact(q, oracle_quantize(x), rows, cols)
+
+
+def test_quantize_static_scale_and_saturation(lib):
+    x = rand_bf16(256, 512, 7)
+    g = np.float32(0.0005)  # small g: many block scales clamp at 448 and many codes at 6
+    q = B.quantize(x.cuda(), g=float(g))
+    ref = oracle_quantize(x, g)
+    assert (ref[1] == 0x7E).any()
+    assert_quant_bitexact(q, ref, 256, 512)
+
+
+def test_quantize_zero_and_tiny_blocks(lib):
+    x = rand_bf16(128, 256, 8)
+    x[3] = 0
+    x[5, :16] = 1e-30
+    x[6] = -x[6].abs()
+    q = B.quantize(x.cuda())
+    assert_quant_bitexact(q, oracle_quantize(x), 128, 256)
+    z = torch.zeros(64, 64, dtype=torch.bfloat16)
+    qz = B.quantize(z.cuda())
+    assert qz.g.item() == 1.0
+    assert_quant_bitexact(qz, oracle_quantize(z), 64, 64)
+
+
+def test_quantize_strided_input(lib):
+    x = rand_bf16(70, 1024, 9)
+    xs = x.cuda()[:, 256:768]
+    assert xs.stride(0) == 1024
+    q = B.quantize(xs)
+    assert_quant_bitexact(q, oracle_quantize(x[:, 256:768].contiguous()), 70, 512)
+
+
+def test_amax(lib):
+    x = rand_bf16(513, 4608, 10, dist="t")
+    got = B.amax(x.cuda()).item()
+    assert got == float(np.max(np.abs(f32(x))))
+    xs = x.cuda()[:, :2304]
+    assert B.amax(xs).item() == float(np.max(np.abs(f32(x[:, :2304]))))
+
+
+@pytest.mark.parametrize("rows,cols,seed", [(130, 208, 11), (256, 4608, 12)])
+def test_dequantize_bitexact(lib, rows, cols, seed):
+    x = rand_bf16(rows, cols, seed)
+    q = B.quantize(x.cuda())
+    got = B.dequantize(q)
+    c, s, g = oracle_quantize(x)
+    want = O.to_bf16_round(O.dequantize(c, s, g))
+    np.testing.assert_array_equal(f32(got), want)
+    B.check_device_error()
+
+
+@pytest.mark.parametrize("name", ["tiny", "qkv_x", "qkv_w", "text_x", "text_w"])
+def test_quantize_bitexact_workload_tensors(lib, name):
+    if name == "tiny":
+        case = W.tiny()
+        tensors = [case.x, case.w]
+    elif name.startswith("qkv"):
+        case = W.qkv_1k()
+        tensors = [case.x if name == "qkv_x" else case.w]
+    else:
+        case = W.text_proj(W.PROMPT_T)
+        tensors = [case.x if name == "text_x" else case.w]
+    for t in tensors:
+        q = B.quantize(t.cuda())
+        assert_quant_bitexact(q, oracle_quantize(t), *t.shape)
