@@ -75,14 +75,16 @@ int64_t k_atoms_of(int64_t cols) { return (cols / 16 + 3) / 4; }
 
 int64_t ld_codes_of(const nvfp4_tensor* t) { return t->ld_codes ? t->ld_codes : t->cols / 2; }
 
-// Checks shared by every NVFP4 tensor argument.
-nvfp4_status check_tensor(const nvfp4_tensor* t, bool need_scale) {
+// Checks shared by every NVFP4 tensor argument.  The quantiser and dequantiser move codes in 4- and
+// 8-byte words, so their code rows need 8-byte alignment; the GEMM reads them with TMA (16 bytes).
+nvfp4_status check_tensor(const nvfp4_tensor* t, bool need_scale, int64_t ld_align) {
   if (!t || !t->codes || !t->scales || (need_scale && !t->tensor_scale)) return NVFP4_ERR_INVALID_ARG;
   if (t->rows < 0 || t->cols <= 0) return NVFP4_ERR_INVALID_ARG;
   if (t->cols % 16) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   const int64_t ld = ld_codes_of(t);
   if (ld < t->cols / 2) return NVFP4_ERR_INVALID_ARG;
-  if (!aligned16(t->codes) || (ld % 16) || !aligned16(t->scales) || (t->tensor_scale && !aligned4(t->tensor_scale)))
+  if (!aligned16(t->codes) || (ld % ld_align) || !aligned16(t->scales) ||
+      (t->tensor_scale && !aligned4(t->tensor_scale)))
     return NVFP4_ERR_MISALIGNED;
   return NVFP4_OK;
 }
@@ -184,7 +186,7 @@ nvfp4_status nvfp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ldx, 
 nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int32_t compute_scale,
                             const nvfp4_tensor* out, nvfp4_stream_t stream) {
   if (!x || !out || rows < 0 || cols <= 0 || ldx < cols) return NVFP4_ERR_INVALID_ARG;
-  if (nvfp4_status e = check_tensor(out, true)) return e;
+  if (nvfp4_status e = check_tensor(out, true, 8)) return e;
   if (out->rows != rows || out->cols != cols) return NVFP4_ERR_INVALID_ARG;
   if (!aligned16(x) || (ldx * 2) % 16) return NVFP4_ERR_MISALIGNED;
   DeviceState* st;
@@ -212,7 +214,7 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
 
 nvfp4_status nvfp4_dequantize(const nvfp4_tensor* t, void* out_bf16, int64_t ld_out, nvfp4_stream_t stream) {
   if (!out_bf16) return NVFP4_ERR_INVALID_ARG;
-  if (nvfp4_status e = check_tensor(t, true)) return e;
+  if (nvfp4_status e = check_tensor(t, true, 8)) return e;
   if (ld_out < t->cols) return NVFP4_ERR_INVALID_ARG;
   if (!aligned16(out_bf16) || (ld_out * 2) % 16) return NVFP4_ERR_MISALIGNED;
   if (t->rows == 0) return NVFP4_OK;
@@ -228,8 +230,8 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor* t, void* out_bf16, int64_t ld_
 nvfp4_status nvfp4_linear(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvfp4_epilogue_desc* epi,
                           void* out_bf16, int64_t ld_out, const nvfp4_tensor* out_fp4, nvfp4_stream_t stream) {
   if (!epi) return NVFP4_ERR_INVALID_ARG;
-  if (nvfp4_status e = check_tensor(a, true)) return e;
-  if (nvfp4_status e = check_tensor(w, true)) return e;
+  if (nvfp4_status e = check_tensor(a, true, 16)) return e;
+  if (nvfp4_status e = check_tensor(w, true, 16)) return e;
   const int64_t M = a->rows, N = w->rows, K = a->cols;
   if (w->cols != K) return NVFP4_ERR_INVALID_ARG;
   if (epi->kind < NVFP4_EPI_BIAS || epi->kind > NVFP4_EPI_RESID_GATE) return NVFP4_ERR_INVALID_ARG;
@@ -250,7 +252,7 @@ nvfp4_status nvfp4_linear(const nvfp4_tensor* a, const nvfp4_tensor* w, const nv
     if (!aligned16(epi->residual) || (epi->ld_residual * 2) % 16 || !aligned16(epi->gate)) return NVFP4_ERR_MISALIGNED;
   }
   if (epi->out_nvfp4) {
-    if (nvfp4_status e = check_tensor(out_fp4, true)) return e;
+    if (nvfp4_status e = check_tensor(out_fp4, true, 16)) return e;
     if (out_fp4->rows != M || out_fp4->cols != n_out) return NVFP4_ERR_INVALID_ARG;
   } else if (!out_bf16) {
     return NVFP4_ERR_INVALID_ARG;

@@ -60,8 +60,9 @@ typedef enum {
  * An NVFP4 tensor of `rows` x `cols` logical elements (cols = the reduction dimension K for GEMM
  * operands).
  *   codes:        uint8, row r starts at codes + r * ld_codes; element k of the row is the low nibble
- *                 of byte k/2 when k is even, the high nibble when k is odd.  ld_codes >= cols/2 and a
- *                 multiple of 16 (0 means cols/2).
+ *                 of byte k/2 when k is even, the high nibble when k is odd.  ld_codes >= cols/2
+ *                 (0 means cols/2); a multiple of 8 for nvfp4_quantize / nvfp4_dequantize and of 16
+ *                 for the operands and the NVFP4 output of nvfp4_linear.
  *   scales:       uint8 E4M3 block scales in the tensor-core scale layout, nvfp4_scale_bytes(rows, cols)
  *                 bytes: 512-byte atoms of 128 rows x 4 blocks, atoms ordered along K first, then along
  *                 rows; inside an atom row r, block c is at (r%32)*16 + ((r/32)%4)*4 + c%4 (see
@@ -121,8 +122,8 @@ typedef struct {
  *   compute_scale = 1: compute g = amax(|x|) / 2688 on the device and store it in *out->tensor_scale
  *                      (an amax pass, the quantise pass and a one-thread finalise, stream-ordered).
  *   compute_scale = 0: use the g already stored in *out->tensor_scale (a calibrated static scale).
- * Rules: cols % 16 == 0; x and ldx*2 16-byte aligned; codes and ld_codes 16-byte aligned; scales
- * 16-byte aligned.  rows == 0 is a no-op.
+ * Rules: cols % 16 == 0; x, ldx*2, codes and scales 16-byte aligned; ld_codes a multiple of 8.
+ * rows == 0 is a no-op.
  */
 NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int32_t compute_scale,
                             const nvfp4_tensor* out, nvfp4_stream_t stream);
