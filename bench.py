@@ -381,15 +381,96 @@ def run_reference(args, ws, rank):
             "e2e": {"value": round(val, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ------------------------------------------------------------------------------------------
+# single-op mode: one layer of one workload, for per-config numbers and profiler captures
+# ------------------------------------------------------------------------------------------
+
+def op_case(name):
+    """(description, setup) for one op; setup() returns a zero-argument callable running the op once
+    (through the C ABI) and the op's algorithmic FLOPs or bytes."""
+    from epilogue_gemm_nvfp4_b200 import binding as B
+    dev = torch.device("cuda")
+
+    def gemm(case, requant=False):
+        a = B.quantize(case.x.to(dev))
+        w = B.quantize(case.w.to(dev))
+        bias = case.bias.to(dev) if case.bias is not None else None
+        ex = {}
+        if case.epilogue == "qknorm":
+            e = case.extras
+            ex = dict(gamma_q=e["gamma_q"].to(dev), gamma_k=e["gamma_k"].to(dev), eps=e["eps"], q_col0=e["q_col0"],
+                      k_col0=e["k_col0"], qk_cols=e["qk_cols"], head_dim=e["head_dim"])
+        elif case.epilogue == "resid_gate":
+            ex = dict(residual=case.extras["residual"].to(dev), gate=case.extras["gate"].to(dev))
+        q = None
+        if requant:
+            q = B.QTensor.empty(case.M, case.n_out)
+            q.g.fill_(0.01)
+        out = torch.empty(case.M, case.n_out, dtype=torch.bfloat16, device=dev)
+        fn = lambda: B.linear(a, w, case.epilogue, bias=bias, out=out if q is None else None, out_fp4=q,
+                              want_bf16=q is None, **ex)
+        return fn, W.flops(case), "TFLOP/s"
+
+    def quant(rows, cols):
+        x = W.to_bf16(W.normal(np.random.default_rng(0), (rows, cols))).to(dev)
+        q = B.QTensor.empty(rows, cols)
+        return (lambda: B.quantize(x, out=q)), 2.5625 * rows * cols, "GB/s (2.5625 B/elem)"
+
+    M1 = W.IMG_TOKENS_1K + W.PROMPT_T
+    M2 = W.IMG_TOKENS_2K + W.PROMPT_T
+    table = {
+        "tiny": lambda: gemm(W.tiny()),
+        "qkv_1k": lambda: gemm(W.qkv_1k()),
+        "up_1k": lambda: gemm(W.case_ffn_up(M1), requant=True),
+        "down_1k": lambda: gemm(W.case_ffn_down(M1)),
+        "text_512": lambda: gemm(W.text_proj(W.PROMPT_T)),
+        "text_1941": lambda: gemm(W.text_proj(W.LONG_PROMPT_T)),
+        "text_512z": lambda: gemm(W.text_proj(W.PROMPT_T, zero_rows=W.IMG_TOKENS_1K)),
+        "out_2k": lambda: gemm(W.case_bias(M2, W.HIDDEN, W.HIDDEN, seed=8, w_std=0.015)),
+        "quant_1k": lambda: quant(M1, W.HIDDEN),
+        "quant_2k": lambda: quant(M2, W.HIDDEN),
+        "quant_text": lambda: quant(W.HIDDEN, W.TEXT_K),
+    }
+    return table[name]
+
+
+def run_op(args):
+    from epilogue_gemm_nvfp4_b200 import binding as B
+    torch.cuda.set_device(0)
+    fn, work, unit = op_case(args.op)()
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    B.check_device_error()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for s, e in evs:
+        s.record()
+        fn()
+        e.record()
+    torch.cuda.synchronize()
+    B.check_device_error()
+    t = sorted(s.elapsed_time(e) for s, e in evs)
+    med = t[len(t) // 2]
+    scale = 1e12 if unit.startswith("TFLOP") else 1e9
+    return {"op": args.op, "median_us": round(med * 1e3, 2), "min_us": round(t[0] * 1e3, 2),
+            "value": round(work / (med * 1e-3) / scale, 1), "unit": unit, "steps": args.steps}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("native", "reference"), default="native")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default=None, help="time one op instead of the block step (profiling / per-config)")
     args = ap.parse_args()
+    if args.op is not None:
+        for name in args.op.split(","):
+            args.op = name
+            print(json.dumps(run_op(args)), flush=True)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

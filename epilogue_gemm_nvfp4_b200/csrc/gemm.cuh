@@ -1,19 +1,26 @@
 // Block-scaled NVFP4 GEMM with the DiT's follow-on ops fused into the epilogue, for sm_100a.
 //
-// One persistent CTA per SM walks output tiles of 128 rows x BN weight rows.  Warp roles:
-//   warp 0      TMA producer: A/B code tiles (128-byte swizzle) and their scale atoms into a ring of
-//               shared-memory stages, completion counted on the stage's "full" mbarrier.
-//   warp 1      MMA issuer (one thread): per stage, tcgen05.cp of the scale atoms into a TMEM slot
-//               owned by that stage, then four tcgen05.mma.kind::mxf4nvf4 (K = 64 each) accumulating
-//               in TMEM; tcgen05.commit frees the stage and, after the last K step, publishes the
-//               accumulator to the epilogue.
-//   warp 2      TMEM allocation / release.
-//   warps 4..7  epilogue: thread i of warp 4+q owns accumulator row 32q+i (TMEM lane = row), so every
-//               row-wise reduction (the 256-wide head RMSNorm, the 16-element requant blocks) is
-//               thread-local: a 256-column tile holds a whole head, there is no cross-fragment
-//               exchange and no revisit of the output.
-// The per-stage scale slots in TMEM are safe to overwrite without extra waits: the producer only
-// refills stage s after the commit of the MMAs that read stage s (and so its TMEM scale slot).
+// One persistent CTA per SM walks output tiles of 128 rows x BN weight rows (512 threads):
+//   warp 0        TMA producer: A/B code tiles (128-byte swizzle) and their scale atoms into a ring of
+//                 shared-memory stages; completion counted on the stage's `full` mbarrier.
+//   warp 1        MMA issuer (one thread): four tcgen05.mma.kind::mxf4nvf4 (K = 64 each) per stage,
+//                 accumulating in TMEM; tcgen05.commit frees the stage (`empty`) and, after the last
+//                 K step of a tile, hands the accumulator to the epilogue (`acc_full`).
+//   warp 2        TMEM allocation / release.
+//   warps 4..7    scale stagers: move each stage's scale atoms from shared memory into that stage's
+//                 TMEM scale slot with tcgen05.st (replicated into the four 32-lane sub-partitions the
+//                 MMA reads), then arrive on `sf_full`.  This keeps scale traffic off the tensor pipe.
+//   warps 8..15   epilogue, two warpgroups over the same 128 rows: thread i of warp 8+4e+q owns
+//                 accumulator row 32q+i (TMEM lane = row) and half of the tile's columns.  It copies its
+//                 columns into registers, releases TMEM at once (`acc_empty`) so the next tile's MMAs
+//                 start, then applies bias / head RMSNorm / gated SiLU / residual+gate and the NVFP4
+//                 requantisation from registers.  Row-wise reductions are thread-local: the 256-wide
+//                 head's sum of squares reads the other half straight from TMEM before the release, so
+//                 there is no cross-fragment exchange and no revisit of the output.
+//                 Stores go through a 1 KB per-warp shared-memory transpose so that each st.global
+//                 writes whole 32-byte row segments.
+// The per-stage TMEM scale slot is safe to rewrite without extra waits: the producer refills stage s
+// only after the commit of the MMAs that read stage s.
 #pragma once
 
 #include "ptx.cuh"
@@ -56,6 +63,7 @@ struct GemmArgs {
 template <int BN>
 struct GemmCfg {
   static constexpr int BM = 128;
+  static constexpr int THREADS = 512;
   static constexpr int BK_BYTES = 128;                  // 256 E2M1 elements per stage and row
   static constexpr int KSTEPS = 4;                      // MMAs of K = 64 per stage
   static constexpr int A_BYTES = BM * BK_BYTES;
@@ -70,12 +78,15 @@ struct GemmCfg {
   static constexpr int SFB_COLS = KSTEPS * (BN / 32);
   static constexpr int SF_COLS = SFA_COLS + SFB_COLS;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int XPOSE_BYTES = 1024;              // per epilogue warp: 32 rows x 32 bytes
+  static constexpr int AUX_BYTES = 512;                 // barriers and flags
+  static constexpr int SMEM_BYTES = AUX_BYTES + 1023 + STAGES * STAGE_BYTES + EPI_WARPS * XPOSE_BYTES;
   static constexpr uint32_t IDESC = idesc_nvf4(BM, BN);
   static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");
+  static_assert(SF_COLS % 16 == 0, "scale slot is written 16 columns at a time");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area");
+  static_assert((3 * STAGES + 5) * 8 + 16 <= AUX_BYTES, "barrier area");
 };
 
 __device__ __forceinline__ void raise_device_error(unsigned int* word, unsigned int code, volatile int* abort) {
@@ -91,10 +102,10 @@ __device__ __forceinline__ int b_row0(const GemmArgs& a, int nb, int j) {
   return nb * BN + j * 128;
 }
 
-__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* p, float (&f)[32]) {
+__device__ __forceinline__ void load_bf16x16(const __nv_bfloat16* p, float (&f)[16]) {
   const uint4* q = reinterpret_cast<const uint4*>(p);
 #pragma unroll
-  for (int v = 0; v < 4; ++v) {
+  for (int v = 0; v < 2; ++v) {
     const uint4 u = __ldg(q + v);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -110,22 +121,50 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
          (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
 }
 
-// Write 32 consecutive output values of one row: bf16 (RNE) and, when requested, their NVFP4
-// re-quantisation with the caller's tensor scale (the quantiser's block rule applied to the
-// bf16-rounded values).  Rows past M write nothing except zero scales in the padding rows.
-__device__ __forceinline__ void emit_row32(const GemmArgs& a, int row, int col0, const float (&o)[32], float qg) {
+__device__ __forceinline__ void tmem_load32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  tmem_ld_32x32b_x32(taddr, r);
+  tmem_ld_wait();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Write 16 bf16 values of this lane's row at column col0 through the warp's transpose buffer: each
+// lane puts its 32-byte row segment into shared memory, then lane pairs store whole segments of
+// 16 rows per st.global.  Rows at or past M are skipped.
+__device__ __forceinline__ void store_row16_bf16(const GemmArgs& a, uint8_t* xpose, int row0, int col0,
+                                                 const uint32_t* w) {
+  const int lane = threadIdx.x & 31;
+  const int sw = (lane >> 2) & 1;  // the two 16-byte halves swap every 4 rows: no bank conflicts
+  uint4* mine = reinterpret_cast<uint4*>(xpose + lane * 32);
+  mine[sw] = make_uint4(w[0], w[1], w[2], w[3]);
+  mine[sw ^ 1] = make_uint4(w[4], w[5], w[6], w[7]);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int r = 16 * i + (lane >> 1), c = lane & 1;
+    const uint4 v = *reinterpret_cast<const uint4*>(xpose + r * 32 + ((c ^ ((r >> 2) & 1)) * 16));
+    if (row0 + r < a.M)
+      *reinterpret_cast<uint4*>(a.out + static_cast<int64_t>(row0 + r) * a.ld_out + col0 + c * 8) = v;
+  }
+  __syncwarp();
+}
+
+// 32 consecutive output values of one row: bf16 (RNE) output and, when requested, the NVFP4
+// re-quantisation of those bf16 values with the caller's tensor scale (the quantiser's block rule).
+__device__ __forceinline__ void emit_row32(const GemmArgs& a, uint8_t* xpose, int row0, int row, int col0,
+                                           const float* o, float qg) {
   uint32_t packed[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(o[2 * i], o[2 * i + 1]);
-  if (row < a.M && a.out != nullptr) {
-    uint4* dst = reinterpret_cast<uint4*>(a.out + static_cast<int64_t>(row) * a.ld_out + col0);
-#pragma unroll
-    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+  if (a.out != nullptr) {
+    store_row16_bf16(a, xpose, row0, col0, packed);
+    store_row16_bf16(a, xpose, row0, col0 + 16, packed + 8);
   }
   if (a.q_codes != nullptr) {
     const int64_t soff = scale_offset(row, col0 / 16, a.q_k_atoms);
     if (row >= a.M) {
-      *reinterpret_cast<uint16_t*>(a.q_scales + soff) = 0;
+      *reinterpret_cast<uint16_t*>(a.q_scales + soff) = 0;  // padding rows of the scale layout
       return;
     }
     uint32_t words[4];
@@ -157,121 +196,150 @@ __device__ __forceinline__ void emit_row32(const GemmArgs& a, int row, int col0,
   }
 }
 
-__device__ __forceinline__ void tmem_load_f32x32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  tmem_ld_32x32b_x32(taddr, r);
-  tmem_ld_wait();
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
+// ------------------------------------------------------------------------------------------
+// epilogue: registers <- TMEM, release, then math and stores
+// ------------------------------------------------------------------------------------------
 
-// Epilogue for one tile; t_acc addresses this warp's 32 lanes at the tile's first column.
 template <int BN, int KIND>
-__device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t t_acc, int row, int nb, float alpha,
-                                              float qg) {
-  if constexpr (KIND == kEpiGatedSilu) {
-    static_assert(BN == 256, "gated SiLU pairs two 128-row weight boxes");
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      const int ocol = nb * 128 + c * 32;
-      float ya[32], yb[32];
-      tmem_load_f32x32(t_acc + c * 32, ya);
-      tmem_load_f32x32(t_acc + 128 + c * 32, yb);
+struct Epilogue {
+  static constexpr int COLS = (KIND == kEpiGatedSilu) ? 128 : BN / 2;  // accumulator columns per thread
+
+  // Copy this thread's accumulator columns into `acc`; for the head RMSNorm also return the sum of
+  // squares of the whole biased 256-wide row (the other half is read from TMEM and dropped).
+  static __device__ __forceinline__ void load(const GemmArgs& a, uint32_t t_acc, int e, int nb, float alpha,
+                                              bool norm, float* acc, float& ss) {
+    if constexpr (KIND == kEpiGatedSilu) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) { ya[i] *= alpha; yb[i] *= alpha; }
-      if (a.bias != nullptr) {
-        float ba[32], bb[32];
-        load_bf16x32(a.bias + ocol, ba);
-        load_bf16x32(a.bias + a.N / 2 + ocol, bb);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) { ya[i] += ba[i]; yb[i] += bb[i]; }
+      for (int c = 0; c < 2; ++c) {
+        tmem_load32(t_acc + 64 * e + 32 * c, acc + 32 * c);              // a
+        tmem_load32(t_acc + 128 + 64 * e + 32 * c, acc + 64 + 32 * c);   // b
       }
-      float o[32];
+    } else {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) o[i] = ya[i] / (1.0f + __expf(-ya[i])) * yb[i];
-      emit_row32(a, row, ocol, o, qg);
-    }
-  } else {
-    const int col_base = nb * BN;
-    const __nv_bfloat16* gamma = nullptr;
-    if constexpr (KIND == kEpiQkNorm) {
-      if (col_base >= a.q_col0 && col_base < a.q_col0 + a.qk_cols) gamma = a.gamma_q;
-      else if (col_base >= a.k_col0 && col_base < a.k_col0 + a.qk_cols) gamma = a.gamma_k;
-    }
-    float rs = 1.0f;
-    if (KIND == kEpiQkNorm && gamma != nullptr) {
-      // pass 1 over TMEM: sum of squares of the biased head (the tile is exactly one 256-wide head)
-      float ss = 0.0f;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        float y[32];
-        tmem_load_f32x32(t_acc + c * 32, y);
-        float b[32];
-        if (a.bias != nullptr) load_bf16x32(a.bias + col_base + c * 32, b);
+      for (int c = 0; c < COLS / 32; ++c) tmem_load32(t_acc + COLS * e + 32 * c, acc + 32 * c);
+      if constexpr (KIND == kEpiQkNorm) {
+        ss = 0.0f;
+        if (norm) {
+          const int col_base = nb * BN;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float v = y[i] * alpha + (a.bias != nullptr ? b[i] : 0.0f);
-          ss = fmaf(v, v, ss);
+          for (int half = 0; half < 2; ++half) {
+#pragma unroll
+            for (int g = 0; g < COLS / 16; ++g) {
+              float other[16];
+              if (half != e) {
+                uint32_t r[16];
+                tmem_ld_32x32b_x16(t_acc + COLS * half + 16 * g, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) other[i] = __uint_as_float(r[i]);
+              }
+              float b[16];
+              if (a.bias != nullptr) load_bf16x16(a.bias + col_base + COLS * half + 16 * g, b);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float raw = (half != e) ? other[i] : acc[16 * g + i];
+                const float v = raw * alpha + (a.bias != nullptr ? b[i] : 0.0f);
+                ss = fmaf(v, v, ss);
+              }
+            }
+          }
         }
       }
-      rs = rsqrtf(ss * (1.0f / BN) + a.eps);
-    }
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      const int col0 = col_base + c * 32;
-      float y[32];
-      tmem_load_f32x32(t_acc + c * 32, y);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) y[i] *= alpha;
-      if (a.bias != nullptr) {
-        float b[32];
-        load_bf16x32(a.bias + col0, b);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) y[i] += b[i];
-      }
-      if (KIND == kEpiQkNorm && gamma != nullptr) {
-        float gm[32];
-        load_bf16x32(gamma + c * 32, gm);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) y[i] = y[i] * rs * gm[i];
-      }
-      if constexpr (KIND == kEpiResidGate) {
-        float r[32];
-        if (row < a.M) load_bf16x32(a.residual + static_cast<int64_t>(row) * a.ld_res + col0, r);
-        else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = 0.0f;
-        }
-        const float4* gp = reinterpret_cast<const float4*>(a.gate + col0);
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const float4 gg = __ldg(gp + v);
-          y[4 * v + 0] = fmaf(gg.x, y[4 * v + 0], r[4 * v + 0]);
-          y[4 * v + 1] = fmaf(gg.y, y[4 * v + 1], r[4 * v + 1]);
-          y[4 * v + 2] = fmaf(gg.z, y[4 * v + 2], r[4 * v + 2]);
-          y[4 * v + 3] = fmaf(gg.w, y[4 * v + 3], r[4 * v + 3]);
-        }
-      }
-      emit_row32(a, row, col0, y, qg);
     }
   }
-}
+
+  static __device__ __forceinline__ void finish(const GemmArgs& a, uint8_t* xpose, int row0, int row, int e, int nb,
+                                                float alpha, float qg, const __nv_bfloat16* gamma, float ss,
+                                                float* acc) {
+    if constexpr (KIND == kEpiGatedSilu) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int ocol = nb * 128 + 64 * e + 32 * c;
+        float o[32];
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          float ba[16], bb[16];
+          if (a.bias != nullptr) {
+            load_bf16x16(a.bias + ocol + 16 * g, ba);
+            load_bf16x16(a.bias + a.N / 2 + ocol + 16 * g, bb);
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float ya = acc[32 * c + 16 * g + i] * alpha, yb = acc[64 + 32 * c + 16 * g + i] * alpha;
+            if (a.bias != nullptr) {
+              ya += ba[i];
+              yb += bb[i];
+            }
+            o[16 * g + i] = ya / (1.0f + __expf(-ya)) * yb;
+          }
+        }
+        emit_row32(a, xpose, row0, row, ocol, o, qg);
+      }
+    } else {
+      const int col_e = nb * BN + COLS * e;
+      float rs = 1.0f;
+      if (KIND == kEpiQkNorm && gamma != nullptr) rs = rsqrtf(ss * (1.0f / BN) + a.eps);
+#pragma unroll
+      for (int c = 0; c < COLS / 32; ++c) {
+        const int col0 = col_e + 32 * c;
+        float* y = acc + 32 * c;
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          float b[16];
+          if (a.bias != nullptr) load_bf16x16(a.bias + col0 + 16 * g, b);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) y[16 * g + i] = y[16 * g + i] * alpha + (a.bias != nullptr ? b[i] : 0.0f);
+          if (KIND == kEpiQkNorm && gamma != nullptr) {
+            float gm[16];
+            load_bf16x16(gamma + COLS * e + 32 * c + 16 * g, gm);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) y[16 * g + i] = y[16 * g + i] * rs * gm[i];
+          }
+          if constexpr (KIND == kEpiResidGate) {
+            float r[16];
+            if (row < a.M) {
+              load_bf16x16(a.residual + static_cast<int64_t>(row) * a.ld_res + col0 + 16 * g, r);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) r[i] = 0.0f;
+            }
+            const float4* gp = reinterpret_cast<const float4*>(a.gate + col0 + 16 * g);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const float4 gg = __ldg(gp + v);
+              y[16 * g + 4 * v + 0] = fmaf(gg.x, y[16 * g + 4 * v + 0], r[4 * v + 0]);
+              y[16 * g + 4 * v + 1] = fmaf(gg.y, y[16 * g + 4 * v + 1], r[4 * v + 1]);
+              y[16 * g + 4 * v + 2] = fmaf(gg.z, y[16 * g + 4 * v + 2], r[4 * v + 2]);
+              y[16 * g + 4 * v + 3] = fmaf(gg.w, y[16 * g + 4 * v + 3], r[4 * v + 3]);
+            }
+          }
+        }
+        emit_row32(a, xpose, row0, row, col0, y, qg);
+      }
+    }
+  }
+};
 
 template <int BN, int KIND>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(512, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ GemmArgs args) {
   using C = GemmCfg<BN>;
+  using E = Epilogue<BN, KIND>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  // small state first, then the 1024-aligned stage ring (128-byte swizzle atoms), then the transposes
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* sf_full = empty + C::STAGES;
+  uint64_t* acc_full = sf_full + C::STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* never_abort = abort_flag + 1;  // stays 0: drains must not be cut short by an abort
+  uint8_t* ring = smem_raw + C::AUX_BYTES;
+  ring += (1024u - (smem_u32(ring) & 1023u)) & 1023u;
+  uint8_t* xpose_all = ring + C::STAGES * C::STAGE_BYTES;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -280,10 +348,11 @@ __global__ void __launch_bounds__(256, 1)
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_full[s], 4);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], C::EPI_WARPS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -304,126 +373,197 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int num_kb = (args.k_steps + C::KSTEPS - 1) / C::KSTEPS;
 
-  if (warp == 0) {
-    if (lane == 0) {
-    // ------------------------------------------------------------------ TMA producer
+  if (warp < 4) {
+    regs_decrease<56>();
+    if (warp == 0) {
+      if (lane == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t armed_mask = 0, armed_parity = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
+          const int mb = tile % args.num_m_blocks, nb = tile / args.num_m_blocks;
+          for (int kb = 0; kb < num_kb; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            const int ks = min(C::KSTEPS, args.k_steps - kb * C::KSTEPS);
+            const uint32_t sf_bytes = static_cast<uint32_t>(ks) * 512u;
+            mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + sf_bytes * (1 + BN / 128));
+            uint8_t* sa = ring + stage * C::STAGE_BYTES;
+            uint8_t* sb = sa + C::A_BYTES;
+            uint8_t* ssfa = sb + C::B_BYTES;
+            uint8_t* ssfb = ssfa + C::SFA_BYTES;
+            tma_load_2d(sa, &tmap_a, &full[stage], kb * C::BK_BYTES, mb * C::BM);
+#pragma unroll
+            for (int j = 0; j < BN / 128; ++j)
+              tma_load_2d(sb + j * 128 * C::BK_BYTES, &tmap_b, &full[stage], kb * C::BK_BYTES,
+                          b_row0<BN, KIND>(args, nb, j));
+            bulk_load(ssfa, args.sfa + (static_cast<int64_t>(mb) * args.k_atoms + kb * 4) * 512, sf_bytes,
+                      &full[stage]);
+#pragma unroll
+            for (int j = 0; j < BN / 128; ++j)
+              bulk_load(ssfb + j * 2048,
+                        args.sfb + (static_cast<int64_t>(b_row0<BN, KIND>(args, nb, j) / 128) * args.k_atoms +
+                                    kb * 4) * 512,
+                        sf_bytes, &full[stage]);
+            armed_mask |= 1u << stage;
+            armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+            if (++stage == C::STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+        if (!ok) raise_device_error(args.error_word, kErrTimeout, abort_flag);
+        // every copy this thread started must land before the CTA's shared memory is released
+        for (int s = 0; s < C::STAGES; ++s)
+          if (armed_mask & (1u << s)) mbar_wait(&full[s], (armed_parity >> s) & 1u, never_abort, args.timeout_ns);
+      }
+      __syncwarp();
+    } else if (warp == 1) {
+      if (lane == 0) {
+        // ---------------------------------------------------------------- MMA issuer
+        int stage = 0;
+        uint32_t phase = 0;
+        int abuf = 0;
+        uint32_t aphase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
+          if (!mbar_wait(&acc_empty[abuf], aphase ^ 1u, abort_flag, args.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * BN);
+          for (int kb = 0; kb < num_kb; ++kb) {
+            if (!mbar_wait(&sf_full[stage], phase, abort_flag, args.timeout_ns) ||
+                !mbar_wait(&full[stage], phase, abort_flag, args.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const int ks = min(C::KSTEPS, args.k_steps - kb * C::KSTEPS);
+            const uint32_t a_addr = smem_u32(ring + stage * C::STAGE_BYTES);
+            const uint32_t b_addr = a_addr + C::A_BYTES;
+            const uint32_t sfa_t = tmem_base + C::SF_COL0 + stage * C::SF_COLS;
+            const uint32_t sfb_t = sfa_t + C::SFA_COLS;
+            for (int k = 0; k < ks; ++k)
+              tc_mma_nvf4(d_tmem, desc_kmajor_sw128(a_addr + k * 32), desc_kmajor_sw128(b_addr + k * 32), C::IDESC,
+                          (kb | k) != 0 ? 1u : 0u, sfa_t + k * 4, sfb_t + k * (BN / 32));
+            tc_commit(&empty[stage]);
+            if (++stage == C::STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (!ok) break;
+          tc_commit(&acc_full[abuf]);
+          if (++abuf == C::ACC_BUFS) {
+            abuf = 0;
+            aphase ^= 1u;
+          }
+        }
+        if (!ok) raise_device_error(args.error_word, kErrTimeout, abort_flag);
+        // every tcgen05 operation this thread issued must finish before TMEM and smem are released
+        tc_commit(drain);
+        mbar_wait(drain, 0, never_abort, args.timeout_ns);
+      }
+      __syncwarp();
+    }
+  } else if (warp < 8) {
+    regs_decrease<64>();
+    // ------------------------------------------------------------------ scale stagers
+    // Lane i of warp 4+q writes TMEM lane 32q+i.  The MMA reads, for row r of a 128-row block, the
+    // 4 scales of one K step from column r / 32 of that step's group of 4 columns, identically in
+    // every sub-partition; 16-byte row i of a 512-byte scale atom is exactly those 4 columns of lane i.
+    const int q = warp & 3;
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t armed_mask = 0, armed_parity = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
-      const int mb = tile % args.num_m_blocks, nb = tile / args.num_m_blocks;
+    for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x) {
+      bool ok = true;
       for (int kb = 0; kb < num_kb; ++kb) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.timeout_ns)) {
+        const bool got = mbar_wait(&full[stage], phase, abort_flag, args.timeout_ns);
+        if (!__all_sync(0xFFFFFFFFu, got)) {
           ok = false;
           break;
         }
+        const uint8_t* ssfa = ring + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
+        const uint8_t* ssfb = ssfa + C::SFA_BYTES;
         const int ks = min(C::KSTEPS, args.k_steps - kb * C::KSTEPS);
-        const uint32_t sf_bytes = static_cast<uint32_t>(ks) * 512u;
-        mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + sf_bytes * (1 + BN / 128));
-        uint8_t* sa = smem + stage * C::STAGE_BYTES;
-        uint8_t* sb = sa + C::A_BYTES;
-        uint8_t* ssfa = sb + C::B_BYTES;
-        uint8_t* ssfb = ssfa + C::SFA_BYTES;
-        tma_load_2d(sa, &tmap_a, &full[stage], kb * C::BK_BYTES, mb * C::BM);
+        const uint32_t t_sf = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + C::SF_COL0 + stage * C::SF_COLS;
+        // slot column order: A steps 0..3 (4 columns each), then for each step k the weight's
+        // 128-row blocks j = 0 .. BN/128-1 (4 columns each)
+        constexpr int NV = C::SF_COLS / 4;  // 16-byte vectors per lane
 #pragma unroll
-        for (int j = 0; j < BN / 128; ++j)
-          tma_load_2d(sb + j * 128 * C::BK_BYTES, &tmap_b, &full[stage], kb * C::BK_BYTES,
-                      b_row0<BN, KIND>(args, nb, j));
-        bulk_load(ssfa, args.sfa + (static_cast<int64_t>(mb) * args.k_atoms + kb * 4) * 512, sf_bytes, &full[stage]);
+        for (int grp = 0; grp < NV / 4; ++grp) {
+          uint32_t v[16];
 #pragma unroll
-        for (int j = 0; j < BN / 128; ++j)
-          bulk_load(ssfb + j * 2048,
-                    args.sfb + (static_cast<int64_t>(b_row0<BN, KIND>(args, nb, j) / 128) * args.k_atoms + kb * 4) * 512,
-                    sf_bytes, &full[stage]);
-        armed_mask |= 1u << stage;
-        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          for (int u = 0; u < 4; ++u) {
+            const int idx = grp * 4 + u;
+            int k;
+            const uint8_t* src;
+            if (idx < 4) {
+              k = idx;
+              src = ssfa + k * 512;
+            } else {
+              k = (idx - 4) / (BN / 128);
+              src = ssfb + ((idx - 4) % (BN / 128)) * 2048 + k * 512;
+            }
+            uint4 x = make_uint4(0, 0, 0, 0);
+            if (k < ks) x = *reinterpret_cast<const uint4*>(src + lane * 16);
+            v[4 * u + 0] = x.x;
+            v[4 * u + 1] = x.y;
+            v[4 * u + 2] = x.z;
+            v[4 * u + 3] = x.w;
+          }
+          tmem_st_32x32b_x16(t_sf + grp * 16, v);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_full[stage]);
         if (++stage == C::STAGES) {
           stage = 0;
           phase ^= 1u;
         }
       }
-    }
-    if (!ok) raise_device_error(args.error_word, kErrTimeout, abort_flag);
-    // every copy this thread started must land before the CTA's shared memory is released
-    for (int s = 0; s < C::STAGES; ++s)
-      if (armed_mask & (1u << s)) mbar_wait(&full[s], (armed_parity >> s) & 1u, never_abort, args.timeout_ns);
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    if (lane == 0) {
-    // ------------------------------------------------------------------ MMA issuer
-    int stage = 0;
-    uint32_t phase = 0;
-    int abuf = 0;
-    uint32_t aphase = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
-      if (!mbar_wait(&acc_empty[abuf], aphase ^ 1u, abort_flag, args.timeout_ns)) {
-        ok = false;
+      if (!ok) {
+        if (lane == 0) raise_device_error(args.error_word, kErrTimeout, abort_flag);
         break;
       }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * BN);
-      for (int kb = 0; kb < num_kb; ++kb) {
-        if (!mbar_wait(&full[stage], phase, abort_flag, args.timeout_ns)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const int ks = min(C::KSTEPS, args.k_steps - kb * C::KSTEPS);
-        const uint8_t* sa = smem + stage * C::STAGE_BYTES;
-        const uint8_t* sb = sa + C::A_BYTES;
-        const uint8_t* ssfa = sb + C::B_BYTES;
-        const uint8_t* ssfb = ssfa + C::SFA_BYTES;
-        const uint32_t sfa_t = tmem_base + C::SF_COL0 + stage * C::SF_COLS;
-        const uint32_t sfb_t = sfa_t + C::SFA_COLS;
-        for (int k = 0; k < ks; ++k) tc_cp_32x128b_warpx4(sfa_t + k * 4, desc_scale_block(smem_u32(ssfa + k * 512)));
-#pragma unroll
-        for (int j = 0; j < BN / 128; ++j)
-          for (int k = 0; k < ks; ++k)
-            tc_cp_32x128b_warpx4(sfb_t + k * (BN / 32) + j * 4, desc_scale_block(smem_u32(ssfb + j * 2048 + k * 512)));
-        const uint32_t a_addr = smem_u32(sa), b_addr = smem_u32(sb);
-        for (int k = 0; k < ks; ++k)
-          tc_mma_nvf4(d_tmem, desc_kmajor_sw128(a_addr + k * 32), desc_kmajor_sw128(b_addr + k * 32), C::IDESC,
-                      (kb | k) != 0 ? 1u : 0u, sfa_t + k * 4, sfb_t + k * (BN / 32));
-        tc_commit(&empty[stage]);
-        if (++stage == C::STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-      if (!ok) break;
-      tc_commit(&acc_full[abuf]);
-      if (++abuf == C::ACC_BUFS) {
-        abuf = 0;
-        aphase ^= 1u;
-      }
     }
-    if (!ok) raise_device_error(args.error_word, kErrTimeout, abort_flag);
-    // every tcgen05 operation this thread issued must finish before TMEM and smem are released
-    tc_commit(drain);
-    mbar_wait(drain, 0, never_abort, args.timeout_ns);
-    }
-    __syncwarp();
-  } else if (warp >= 4) {
+  } else {
+    regs_increase<192>();
     // ------------------------------------------------------------------ epilogue
+    const int e = (warp - 8) >> 2;
     const int q = warp & 3;
+    uint8_t* xpose = xpose_all + (warp - 8) * C::XPOSE_BYTES;
     const float alpha = __fmul_rn(*args.ga, *args.gb);
     const float qg = args.q_codes != nullptr ? *args.q_g : 1.0f;
     int abuf = 0;
     uint32_t aphase = 0;
     for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x) {
       const int mb = tile % args.num_m_blocks, nb = tile / args.num_m_blocks;
+      const __nv_bfloat16* gamma = nullptr;
+      if constexpr (KIND == kEpiQkNorm) {
+        const int col_base = nb * BN;
+        if (col_base >= args.q_col0 && col_base < args.q_col0 + args.qk_cols) gamma = args.gamma_q;
+        else if (col_base >= args.k_col0 && col_base < args.k_col0 + args.qk_cols) gamma = args.gamma_k;
+      }
       const bool got = mbar_wait(&acc_full[abuf], aphase, abort_flag, args.timeout_ns);
       if (!__all_sync(0xFFFFFFFFu, got)) {  // the tcgen05.ld below needs the whole warp
         if (lane == 0) raise_device_error(args.error_word, kErrTimeout, abort_flag);
         break;
       }
       tc_fence_after();
-      const int row = mb * C::BM + q * 32 + lane;
+      const int row0 = mb * C::BM + q * 32;
       const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(abuf * BN);
-      epilogue_tile<BN, KIND>(args, t_acc, row, nb, alpha, qg);
+      float acc[E::COLS];
+      float ss = 0.0f;
+      E::load(args, t_acc, e, nb, alpha, gamma != nullptr, acc, ss);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[abuf]);
@@ -431,6 +571,7 @@ __global__ void __launch_bounds__(256, 1)
         abuf = 0;
         aphase ^= 1u;
       }
+      E::finish(args, xpose, row0, row0 + lane, e, nb, alpha, qg, gamma, ss, acc);
     }
   }
 

@@ -6,7 +6,7 @@
 #include <cstdlib>
 #include <mutex>
 
-#include "../../include/nvfp4.h"
+#include "nvfp4.h"
 #include "gemm.cuh"
 #include "ptx.cuh"
 #include "quantize.cuh"
@@ -136,7 +136,7 @@ nvfp4_status launch_gemm(DeviceState* st, const CUtensorMap& ma, const CUtensorM
     attr = true;
   }
   const int grid = args.num_tiles < st->sm_count ? args.num_tiles : st->sm_count;
-  kernel<<<grid, 256, C::SMEM_BYTES, stream>>>(ma, mb, args);
+  kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, args);
   return launch_status();
 }
 
