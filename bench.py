@@ -411,10 +411,16 @@ def op_case(name):
                               want_bf16=q is None, **ex)
         return fn, W.flops(case), "TFLOP/s"
 
-    def quant(rows, cols):
+    def quant(rows, cols, static=False):
         x = W.to_bf16(W.normal(np.random.default_rng(0), (rows, cols))).to(dev)
         q = B.QTensor.empty(rows, cols)
-        return (lambda: B.quantize(x, out=q)), 2.5625 * rows * cols, "GB/s (2.5625 B/elem)"
+        q.g.fill_(3.0 / 2688.0)
+        return (lambda: B.quantize(x, out=q, static=static)), 2.5625 * rows * cols, "GB/s (2.5625 B/elem)"
+
+    def amax(rows, cols):
+        x = W.to_bf16(W.normal(np.random.default_rng(0), (rows, cols))).to(dev)
+        o = torch.empty(1, dtype=torch.float32, device=dev)
+        return (lambda: B.amax(x, out=o)), 2.0 * rows * cols, "GB/s (2 B/elem)"
 
     M1 = W.IMG_TOKENS_1K + W.PROMPT_T
     M2 = W.IMG_TOKENS_2K + W.PROMPT_T
@@ -430,6 +436,9 @@ def op_case(name):
         "quant_1k": lambda: quant(M1, W.HIDDEN),
         "quant_2k": lambda: quant(M2, W.HIDDEN),
         "quant_text": lambda: quant(W.HIDDEN, W.TEXT_K),
+        "quant_2k_static": lambda: quant(M2, W.HIDDEN, static=True),
+        "quant_text_static": lambda: quant(W.HIDDEN, W.TEXT_K, static=True),
+        "amax_2k": lambda: amax(M2, W.HIDDEN),
     }
     return table[name]
 
@@ -442,17 +451,21 @@ def run_op(args):
         fn()
     torch.cuda.synchronize()
     B.check_device_error()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for s, e in evs:
+    # back-to-back launches between two events: the host enqueues ahead of the device, so the mean
+    # is the device time per call (per-call events would also count host launch gaps)
+    reps = []
+    for _ in range(3):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record()
-        fn()
+        for _ in range(args.steps):
+            fn()
         e.record()
-    torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        reps.append(s.elapsed_time(e) / args.steps)
     B.check_device_error()
-    t = sorted(s.elapsed_time(e) for s, e in evs)
-    med = t[len(t) // 2]
+    med = sorted(reps)[1]
     scale = 1e12 if unit.startswith("TFLOP") else 1e9
-    return {"op": args.op, "median_us": round(med * 1e3, 2), "min_us": round(t[0] * 1e3, 2),
+    return {"op": args.op, "mean_us": round(med * 1e3, 2), "min_us": round(min(reps) * 1e3, 2),
             "value": round(work / (med * 1e-3) / scale, 1), "unit": unit, "steps": args.steps}
 
 

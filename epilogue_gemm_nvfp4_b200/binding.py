@@ -18,8 +18,8 @@ LIB_PATH = os.path.join(_HERE, "libnvfp4.so")
 
 #: every function the header declares
 EXPORTS = ("nvfp4_quantize", "nvfp4_linear", "nvfp4_dequantize", "nvfp4_amax", "nvfp4_scale_bytes",
-           "nvfp4_scale_offset", "nvfp4_get_device_error", "nvfp4_linear_tile_n", "nvfp4_status_string",
-           "nvfp4_version")
+           "nvfp4_scale_offset", "nvfp4_get_device_error", "nvfp4_linear_tile_n", "nvfp4_linear_split_k",
+           "nvfp4_status_string", "nvfp4_version")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_MISALIGNED, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(6)
 EPI_BIAS, EPI_QKNORM, EPI_GATED_SILU, EPI_RESID_GATE = range(4)
@@ -68,6 +68,7 @@ def load() -> ctypes.CDLL:
         "nvfp4_scale_offset": (I64, [I64, I64, I64]),
         "nvfp4_get_device_error": (I32, [P]),
         "nvfp4_linear_tile_n": (I32, [I64, I64, I32]),
+        "nvfp4_linear_split_k": (I32, [I64, I64, I32]),
         "nvfp4_status_string": (ctypes.c_char_p, [I32]),
         "nvfp4_version": (I32, []),
     }
@@ -134,17 +135,23 @@ def tile_n(N: int, K: int, kind: str) -> int:
     return int(load().nvfp4_linear_tile_n(N, K, EPI_KINDS[kind]))
 
 
+def split_k(N: int, K: int, kind: str) -> int:
+    return int(load().nvfp4_linear_split_k(N, K, EPI_KINDS[kind]))
+
+
 def quantize(x: torch.Tensor, out: QTensor | None = None, g: float | torch.Tensor | None = None,
-             stream=None) -> QTensor:
-    """bf16 [rows, cols] (CUDA) -> NVFP4.  g=None computes the tensor scale on the device; otherwise
-    the given decode scale is used as is."""
+             static: bool = False, stream=None) -> QTensor:
+    """bf16 [rows, cols] (CUDA) -> NVFP4.  By default the tensor scale is computed on the device.
+    With ``g`` the given decode scale is stored in out.g and used; with ``static=True`` the scale
+    already held in out.g is used."""
     assert x.is_cuda and x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     rows, cols = x.shape
     out = QTensor.empty(rows, cols, x.device) if out is None else out
     if g is not None:
         out.g.copy_(torch.as_tensor(g, dtype=torch.float32).reshape(1))
+    compute = g is None and not static
     ct = out.c()
-    _check(load().nvfp4_quantize(_ptr(x), rows, cols, x.stride(0), int(g is None), ctypes.byref(ct),
+    _check(load().nvfp4_quantize(_ptr(x), rows, cols, x.stride(0), int(compute), ctypes.byref(ct),
                                  _stream(stream)), "nvfp4_quantize")
     return out
 

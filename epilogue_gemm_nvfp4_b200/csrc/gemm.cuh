@@ -1,15 +1,17 @@
 // Block-scaled NVFP4 GEMM with the DiT's follow-on ops fused into the epilogue, for sm_100a.
 //
 // One persistent CTA per SM walks output tiles of 128 rows x BN weight rows (512 threads):
-//   warp 0        TMA producer: A/B code tiles (128-byte swizzle) and their scale atoms into a ring of
-//                 shared-memory stages; completion counted on the stage's `full` mbarrier.
+//   warp 0        TMA producer: per stage, first the scale atoms (bulk copies, counted on `sf_landed`),
+//                 then the A/B code tiles (TMA, 128-byte swizzle, counted on `full`), into a ring of
+//                 shared-memory stages.
 //   warp 1        MMA issuer (one thread): four tcgen05.mma.kind::mxf4nvf4 (K = 64 each) per stage,
 //                 accumulating in TMEM; tcgen05.commit frees the stage (`empty`) and, after the last
 //                 K step of a tile, hands the accumulator to the epilogue (`acc_full`).
 //   warp 2        TMEM allocation / release.
 //   warps 4..7    scale stagers: move each stage's scale atoms from shared memory into that stage's
 //                 TMEM scale slot with tcgen05.st (replicated into the four 32-lane sub-partitions the
-//                 MMA reads), then arrive on `sf_full`.  This keeps scale traffic off the tensor pipe.
+//                 MMA reads), then arrive on `sf_full`.  This keeps scale traffic off the tensor pipe,
+//                 and since the atoms land before the code tiles it overlaps their copy.
 //   warps 8..15   epilogue, two warpgroups over the same 128 rows: thread i of warp 8+4e+q owns
 //                 accumulator row 32q+i (TMEM lane = row) and half of the tile's columns.  It copies its
 //                 columns into registers, releases TMEM at once (`acc_empty`) so the next tile's MMAs
@@ -58,7 +60,28 @@ struct GemmArgs {
   int32_t q_k_atoms;
   unsigned int* error_word;
   uint64_t timeout_ns;
+  // split-K: `splits` consecutive work units share one output tile, each summing a contiguous range
+  // of K blocks; the first to finish parks its fp32 partial, the second adds it and runs the epilogue.
+  int32_t splits;
+  int32_t num_units;     // num_tiles * splits
+  float* split_partials; // [num_tiles][2][128][cols per thread] fp32
+  unsigned int* split_flags;  // [num_tiles], zero before the launch
 };
+
+struct WorkUnit {
+  int tile, mb, nb, kb0, kb1;
+};
+
+__device__ __forceinline__ WorkUnit work_unit(const GemmArgs& a, int u, int num_kb) {
+  WorkUnit w;
+  const int split = u % a.splits;
+  w.tile = u / a.splits;
+  w.mb = w.tile % a.num_m_blocks;
+  w.nb = w.tile / a.num_m_blocks;
+  w.kb0 = split * num_kb / a.splits;
+  w.kb1 = (split + 1) * num_kb / a.splits;
+  return w;
+}
 
 template <int BN>
 struct GemmCfg {
@@ -86,7 +109,8 @@ struct GemmCfg {
   static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(SF_COLS % 16 == 0, "scale slot is written 16 columns at a time");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert((3 * STAGES + 5) * 8 + 16 <= AUX_BYTES, "barrier area");
+  static_assert((4 * STAGES + 5) * 8 + 16 <= AUX_BYTES, "barrier area");
+  static_assert(BM == 128, "the split-K partial layout assumes 128 rows per tile");
 };
 
 __device__ __forceinline__ void raise_device_error(unsigned int* word, unsigned int code, volatile int* abort) {
@@ -320,6 +344,56 @@ struct Epilogue {
   }
 };
 
+constexpr unsigned int kSplitReady = 0x100u;
+
+// Split-K hand-off for one tile (two work units).  Returns true when this CTA now holds the full sum
+// in `acc` and must run the epilogue; false when it parked its partial for the other unit (or the
+// wait for the other unit's partial ran out of time).  fp32 addition is commutative, so the sum is
+// the same bits whichever unit finishes first; the split depends on K only, never on M.
+template <int COLS>
+__device__ __forceinline__ bool split_exchange(const GemmArgs& a, int tile, int e, int row_local, float* acc,
+                                               volatile int* role_slot, volatile int* abort_flag) {
+  const int et = threadIdx.x - 256;  // epilogue thread 0..255
+  if (et == 0) *role_slot = static_cast<int>(atomicAdd(&a.split_flags[tile], 1u));
+  named_barrier_sync(1, 256);
+  const int role = *role_slot;
+  float4* part = reinterpret_cast<float4*>(a.split_partials +
+                                           ((static_cast<int64_t>(tile) * 2 + e) * 128 + row_local) * COLS);
+  if ((role & 0xFF) == 0) {
+#pragma unroll
+    for (int i = 0; i < COLS / 4; ++i) part[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+    __threadfence();
+    named_barrier_sync(1, 256);
+    if (et == 0) atomicOr(&a.split_flags[tile], kSplitReady);
+    return false;
+  }
+  if (et == 0) {
+    const uint64_t t0 = global_timer_ns();
+    int ok = 1;
+    while ((atomicAdd(&a.split_flags[tile], 0u) & kSplitReady) == 0) {
+      if (*abort_flag || global_timer_ns() - t0 > a.timeout_ns) {
+        ok = 0;
+        break;
+      }
+      __nanosleep(64);
+    }
+    if (!ok) raise_device_error(a.error_word, kErrTimeout, abort_flag);
+    *role_slot = ok ? 1 : -1;
+  }
+  named_barrier_sync(1, 256);
+  if (*role_slot < 0) return false;
+  __threadfence();
+#pragma unroll
+  for (int i = 0; i < COLS / 4; ++i) {
+    const float4 p = __ldcg(part + i);
+    acc[4 * i] += p.x;
+    acc[4 * i + 1] += p.y;
+    acc[4 * i + 2] += p.z;
+    acc[4 * i + 3] += p.w;
+  }
+  return true;
+}
+
 template <int BN, int KIND>
 __global__ void __launch_bounds__(512, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
@@ -331,12 +405,14 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw);
   uint64_t* empty = full + C::STAGES;
   uint64_t* sf_full = empty + C::STAGES;
-  uint64_t* acc_full = sf_full + C::STAGES;
+  uint64_t* sf_landed = sf_full + C::STAGES;
+  uint64_t* acc_full = sf_landed + C::STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* never_abort = abort_flag + 1;  // stays 0: drains must not be cut short by an abort
+  volatile int* split_role = never_abort + 1;
   uint8_t* ring = smem_raw + C::AUX_BYTES;
   ring += (1024u - (smem_u32(ring) & 1023u)) & 1023u;
   uint8_t* xpose_all = ring + C::STAGES * C::STAGE_BYTES;
@@ -349,6 +425,7 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&sf_full[s], 4);
+      mbar_init(&sf_landed[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -382,33 +459,35 @@ __global__ void __launch_bounds__(512, 1)
         uint32_t phase = 0;
         uint32_t armed_mask = 0, armed_parity = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
-          const int mb = tile % args.num_m_blocks, nb = tile / args.num_m_blocks;
-          for (int kb = 0; kb < num_kb; ++kb) {
+        for (int u = blockIdx.x; ok && u < args.num_units; u += gridDim.x) {
+          const WorkUnit wu = work_unit(args, u, num_kb);
+          const int mb = wu.mb, nb = wu.nb;
+          for (int kb = wu.kb0; kb < wu.kb1; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.timeout_ns)) {
               ok = false;
               break;
             }
             const int ks = min(C::KSTEPS, args.k_steps - kb * C::KSTEPS);
             const uint32_t sf_bytes = static_cast<uint32_t>(ks) * 512u;
-            mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + sf_bytes * (1 + BN / 128));
             uint8_t* sa = ring + stage * C::STAGE_BYTES;
             uint8_t* sb = sa + C::A_BYTES;
             uint8_t* ssfa = sb + C::B_BYTES;
             uint8_t* ssfb = ssfa + C::SFA_BYTES;
-            tma_load_2d(sa, &tmap_a, &full[stage], kb * C::BK_BYTES, mb * C::BM);
-#pragma unroll
-            for (int j = 0; j < BN / 128; ++j)
-              tma_load_2d(sb + j * 128 * C::BK_BYTES, &tmap_b, &full[stage], kb * C::BK_BYTES,
-                          b_row0<BN, KIND>(args, nb, j));
+            mbar_arrive_expect_tx(&sf_landed[stage], sf_bytes * (1 + BN / 128));
             bulk_load(ssfa, args.sfa + (static_cast<int64_t>(mb) * args.k_atoms + kb * 4) * 512, sf_bytes,
-                      &full[stage]);
+                      &sf_landed[stage]);
 #pragma unroll
             for (int j = 0; j < BN / 128; ++j)
               bulk_load(ssfb + j * 2048,
                         args.sfb + (static_cast<int64_t>(b_row0<BN, KIND>(args, nb, j) / 128) * args.k_atoms +
                                     kb * 4) * 512,
-                        sf_bytes, &full[stage]);
+                        sf_bytes, &sf_landed[stage]);
+            mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES);
+            tma_load_2d(sa, &tmap_a, &full[stage], kb * C::BK_BYTES, mb * C::BM);
+#pragma unroll
+            for (int j = 0; j < BN / 128; ++j)
+              tma_load_2d(sb + j * 128 * C::BK_BYTES, &tmap_b, &full[stage], kb * C::BK_BYTES,
+                          b_row0<BN, KIND>(args, nb, j));
             armed_mask |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
             if (++stage == C::STAGES) {
@@ -420,7 +499,10 @@ __global__ void __launch_bounds__(512, 1)
         if (!ok) raise_device_error(args.error_word, kErrTimeout, abort_flag);
         // every copy this thread started must land before the CTA's shared memory is released
         for (int s = 0; s < C::STAGES; ++s)
-          if (armed_mask & (1u << s)) mbar_wait(&full[s], (armed_parity >> s) & 1u, never_abort, args.timeout_ns);
+          if (armed_mask & (1u << s)) {
+            mbar_wait(&sf_landed[s], (armed_parity >> s) & 1u, never_abort, args.timeout_ns);
+            mbar_wait(&full[s], (armed_parity >> s) & 1u, never_abort, args.timeout_ns);
+          }
       }
       __syncwarp();
     } else if (warp == 1) {
@@ -431,14 +513,15 @@ __global__ void __launch_bounds__(512, 1)
         int abuf = 0;
         uint32_t aphase = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
+        for (int u = blockIdx.x; ok && u < args.num_units; u += gridDim.x) {
+          const WorkUnit wu = work_unit(args, u, num_kb);
           if (!mbar_wait(&acc_empty[abuf], aphase ^ 1u, abort_flag, args.timeout_ns)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * BN);
-          for (int kb = 0; kb < num_kb; ++kb) {
+          for (int kb = wu.kb0; kb < wu.kb1; ++kb) {
             if (!mbar_wait(&sf_full[stage], phase, abort_flag, args.timeout_ns) ||
                 !mbar_wait(&full[stage], phase, abort_flag, args.timeout_ns)) {
               ok = false;
@@ -452,7 +535,7 @@ __global__ void __launch_bounds__(512, 1)
             const uint32_t sfb_t = sfa_t + C::SFA_COLS;
             for (int k = 0; k < ks; ++k)
               tc_mma_nvf4(d_tmem, desc_kmajor_sw128(a_addr + k * 32), desc_kmajor_sw128(b_addr + k * 32), C::IDESC,
-                          (kb | k) != 0 ? 1u : 0u, sfa_t + k * 4, sfb_t + k * (BN / 32));
+                          (kb != wu.kb0 || k != 0) ? 1u : 0u, sfa_t + k * 4, sfb_t + k * (BN / 32));
             tc_commit(&empty[stage]);
             if (++stage == C::STAGES) {
               stage = 0;
@@ -482,10 +565,11 @@ __global__ void __launch_bounds__(512, 1)
     const int q = warp & 3;
     int stage = 0;
     uint32_t phase = 0;
-    for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x) {
+    for (int u = blockIdx.x; u < args.num_units; u += gridDim.x) {
+      const WorkUnit wu = work_unit(args, u, num_kb);
       bool ok = true;
-      for (int kb = 0; kb < num_kb; ++kb) {
-        const bool got = mbar_wait(&full[stage], phase, abort_flag, args.timeout_ns);
+      for (int kb = wu.kb0; kb < wu.kb1; ++kb) {
+        const bool got = mbar_wait(&sf_landed[stage], phase, abort_flag, args.timeout_ns);
         if (!__all_sync(0xFFFFFFFFu, got)) {
           ok = false;
           break;
@@ -545,8 +629,9 @@ __global__ void __launch_bounds__(512, 1)
     const float qg = args.q_codes != nullptr ? *args.q_g : 1.0f;
     int abuf = 0;
     uint32_t aphase = 0;
-    for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x) {
-      const int mb = tile % args.num_m_blocks, nb = tile / args.num_m_blocks;
+    for (int u = blockIdx.x; u < args.num_units; u += gridDim.x) {
+      const WorkUnit wu = work_unit(args, u, num_kb);
+      const int mb = wu.mb, nb = wu.nb;
       const __nv_bfloat16* gamma = nullptr;
       if constexpr (KIND == kEpiQkNorm) {
         const int col_base = nb * BN;
@@ -571,6 +656,10 @@ __global__ void __launch_bounds__(512, 1)
         abuf = 0;
         aphase ^= 1u;
       }
+      // (the head norm's sum of squares is taken while loading, so the host never splits QK-norm GEMMs)
+      if (KIND != kEpiQkNorm && args.splits > 1 &&
+          !split_exchange<E::COLS>(args, wu.tile, e, q * 32 + lane, acc, split_role, abort_flag))
+        continue;
       E::finish(args, xpose, row0, row0 + lane, e, nb, alpha, qg, gamma, ss, acc);
     }
   }

@@ -1,10 +1,12 @@
 // Host side of libnvfp4: argument checks, TMA descriptors, tile configuration and launches.
-// The library allocates no memory; the only device state it owns is one sticky error word per
-// device, a module-scope __device__ variable.
+// Device state the library owns: one sticky error word per device (a module-scope __device__
+// variable) and the per-stream split-K scratch of long-K GEMMs.
 #include <cudaTypedefs.h>
 
 #include <cstdlib>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "nvfp4.h"
 #include "gemm.cuh"
@@ -28,6 +30,31 @@ struct DeviceState {
 
 std::mutex g_mutex;
 DeviceState g_devices[kMaxDevices];
+
+// Split-K scratch, one buffer per (device, stream) so that calls on different streams never share
+// it.  Grown on demand; growing frees the old buffer (cudaFree waits for the device).
+struct Scratch {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+std::map<std::pair<int, uintptr_t>, Scratch> g_scratch;
+
+nvfp4_status scratch_for(cudaStream_t s, size_t need, void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  Scratch& w = g_scratch[{dev, reinterpret_cast<uintptr_t>(s)}];
+  if (w.bytes < need) {
+    if (w.ptr != nullptr && cudaFree(w.ptr) != cudaSuccess) return NVFP4_ERR_CUDA;
+    w.ptr = nullptr;
+    w.bytes = 0;
+    const size_t sz = (need + (size_t(16) << 20) - 1) & ~((size_t(16) << 20) - 1);
+    if (cudaMalloc(&w.ptr, sz) != cudaSuccess) return NVFP4_ERR_CUDA;
+    w.bytes = sz;
+  }
+  *out = w.ptr;
+  return NVFP4_OK;
+}
 
 // Per-device set-up, done once with that device current: SM count and the address of the error word.
 nvfp4_status device_state(DeviceState** out) {
@@ -91,9 +118,14 @@ nvfp4_status check_tensor(const nvfp4_tensor* t, bool need_scale, int64_t ld_ali
 
 nvfp4_status launch_status() { return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
 
-int elementwise_grid(int64_t work_items, int items_per_cta, int sm_count) {
+// Grid for a grid-stride kernel: enough CTAs for the work, at most one resident wave.
+template <typename Kernel>
+int resident_grid(Kernel kernel, int threads, int64_t work_items, int items_per_cta, int sm_count) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
   int64_t g = (work_items + items_per_cta - 1) / items_per_cta;
-  const int64_t cap = static_cast<int64_t>(sm_count) * 8;
+  const int64_t cap = static_cast<int64_t>(sm_count) * per_sm;
   if (g > cap) g = cap;
   if (g < 1) g = 1;
   return static_cast<int>(g);
@@ -113,6 +145,11 @@ nvfp4_status make_code_map(CUtensorMap* map, const nvfp4_tensor* t) {
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
+
+// Two-way split of K for long reductions (the 53248-wide text projection): a function of K and the
+// epilogue only, never of M, so every row's arithmetic is the same whatever M is.  The head norm takes
+// its sum of squares while loading the accumulator and is never split.
+int split_k_for(int64_t K, int32_t kind) { return (K >= 32768 && kind != NVFP4_EPI_QKNORM) ? 2 : 1; }
 
 int tile_n_for(int64_t N, int64_t K, int32_t kind) {
   if (K < 64 || K % 64) return 0;
@@ -135,7 +172,7 @@ nvfp4_status launch_gemm(DeviceState* st, const CUtensorMap& ma, const CUtensorM
       return NVFP4_ERR_CUDA;
     attr = true;
   }
-  const int grid = args.num_tiles < st->sm_count ? args.num_tiles : st->sm_count;
+  const int grid = args.num_units < st->sm_count ? args.num_units : st->sm_count;
   kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, args);
   return launch_status();
 }
@@ -168,6 +205,10 @@ int64_t nvfp4_scale_offset(int64_t r, int64_t kb, int64_t cols) { return scale_o
 
 int32_t nvfp4_linear_tile_n(int64_t N, int64_t K, int32_t kind) { return tile_n_for(N, K, kind); }
 
+int32_t nvfp4_linear_split_k(int64_t N, int64_t K, int32_t kind) {
+  return tile_n_for(N, K, kind) ? split_k_for(K, kind) : 0;
+}
+
 nvfp4_status nvfp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ldx, float* amax, nvfp4_stream_t stream) {
   if (!x || !amax || rows < 0 || cols <= 0 || ldx < cols) return NVFP4_ERR_INVALID_ARG;
   if (cols % 8) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -177,7 +218,7 @@ nvfp4_status nvfp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ldx, 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(amax, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
   if (rows == 0) return NVFP4_OK;
-  const int grid = elementwise_grid(rows * cols / 8, 256 * 4, st->sm_count);
+  const int grid = resident_grid(amax_kernel, 256, rows * cols / 8, 256 * 4, st->sm_count);
   amax_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), rows, cols, ldx,
                                    reinterpret_cast<unsigned int*>(amax));
   return launch_status();
@@ -196,18 +237,23 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
   auto* codes = static_cast<uint8_t*>(out->codes);
   auto* scales = static_cast<uint8_t*>(out->scales);
   const int64_t ld = ld_codes_of(out), ka = k_atoms_of(cols);
-  const int64_t tasks = rows * ((cols + 255) / 256) + 1;
-  const int qgrid = elementwise_grid(tasks, 8 * kQuantUnroll, st->sm_count);
+  const int64_t steps = (cols / 16 + 31) / 32;
+  const int64_t tasks = rows * ((steps + kQuantStepsPerTask - 1) / kQuantStepsPerTask) + 1;
+  // one 256-bit load per block when every block starts on a 32-byte boundary
+  const bool vec32 = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx * 2) % 32 == 0;
+  auto qk = compute_scale ? (vec32 ? quantize_kernel<true, true, true> : quantize_kernel<true, true, false>)
+                          : (vec32 ? quantize_kernel<false, false, true> : quantize_kernel<false, false, false>);
+  const int qgrid = resident_grid(qk, 256, tasks, 8, st->sm_count);
   if (compute_scale) {
     if (cudaMemsetAsync(out->tensor_scale, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (rows > 0) {
-      const int agrid = elementwise_grid(rows * cols / 8, 256 * 4, st->sm_count);
+      const int agrid = resident_grid(amax_kernel, 256, rows * cols / 8, 256 * 4, st->sm_count);
       amax_kernel<<<agrid, 256, 0, s>>>(xb, rows, cols, ldx, reinterpret_cast<unsigned int*>(out->tensor_scale));
     }
-    quantize_kernel<true><<<qgrid, 256, 0, s>>>(xb, rows, cols, ldx, out->tensor_scale, codes, ld, scales, ka);
+    qk<<<qgrid, 256, 0, s>>>(xb, rows, cols, ldx, out->tensor_scale, codes, ld, scales, ka);
     finalize_scale_kernel<<<1, 1, 0, s>>>(out->tensor_scale);
   } else {
-    quantize_kernel<false><<<qgrid, 256, 0, s>>>(xb, rows, cols, ldx, out->tensor_scale, codes, ld, scales, ka);
+    qk<<<qgrid, 256, 0, s>>>(xb, rows, cols, ldx, out->tensor_scale, codes, ld, scales, ka);
   }
   return launch_status();
 }
@@ -220,7 +266,7 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor* t, void* out_bf16, int64_t ld_
   if (t->rows == 0) return NVFP4_OK;
   DeviceState* st;
   if (nvfp4_status e = device_state(&st)) return e;
-  const int grid = elementwise_grid(t->rows * (t->cols / 16), 256, st->sm_count);
+  const int grid = resident_grid(dequantize_kernel, 256, t->rows * (t->cols / 16), 256, st->sm_count);
   dequantize_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint8_t*>(t->codes), ld_codes_of(t), static_cast<const uint8_t*>(t->scales), t->tensor_scale,
       t->rows, t->cols, k_atoms_of(t->cols), static_cast<__nv_bfloat16*>(out_bf16), ld_out);
@@ -303,8 +349,20 @@ nvfp4_status nvfp4_linear(const nvfp4_tensor* a, const nvfp4_tensor* w, const nv
   }
   g.error_word = st->error_word;
   g.timeout_ns = wait_timeout_ns();
+  g.splits = split_k_for(K, epi->kind);
+  g.num_units = g.num_tiles * g.splits;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (g.splits > 1) {
+    const int cols_per_thread = epi->kind == NVFP4_EPI_GATED_SILU ? 128 : BN / 2;
+    const size_t flag_bytes = (static_cast<size_t>(g.num_tiles) * 4 + 255) & ~size_t(255);
+    const size_t part_bytes = static_cast<size_t>(g.num_tiles) * 2 * 128 * cols_per_thread * 4;
+    void* ws = nullptr;
+    if (nvfp4_status e = scratch_for(s, flag_bytes + part_bytes, &ws)) return e;
+    g.split_flags = static_cast<unsigned int*>(ws);
+    g.split_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + flag_bytes);
+    if (cudaMemsetAsync(ws, 0, static_cast<size_t>(g.num_tiles) * 4, s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  }
   switch (epi->kind) {
     case NVFP4_EPI_BIAS:
       return BN == 256 ? launch_gemm<256, kEpiBias>(st, ma, mb, g, s) : launch_gemm<128, kEpiBias>(st, ma, mb, g, s);

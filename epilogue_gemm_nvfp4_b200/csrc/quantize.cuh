@@ -101,13 +101,30 @@ __device__ __forceinline__ uint32_t block_scale(float amax_b, float g, float& in
 }
 
 // ------------------------------------------------------------------------------------------
-// quantise.  Warp task = (row, 256-element span).  Lane l holds elements [8l, 8l+8) of the span;
-// lanes 2j and 2j+1 form block j and meet with one shuffle for the block amax.
+// quantise.  Lane l of a warp step owns one 16-element block (32 bytes, one 256-bit load); a warp
+// step covers 32 consecutive blocks of a row and a task up to kQuantStepsPerTask steps of one row.
+// The block rule runs once per block in its own lane; four lanes' scale bytes form one aligned
+// 32-bit word of the scale layout.  With kReverse the tasks run from the end of the tensor
+// backwards, so right after the amax pass (which streams the tensor front to back) the first tasks
+// re-read from L2 what that pass left there.
 // ------------------------------------------------------------------------------------------
 
-constexpr int kQuantUnroll = 4;
+constexpr int kQuantStepsPerTask = 8;   // 8 x 512 elements of one row per warp task
+constexpr int kQuantUnroll = 2;         // 32-byte loads in flight per lane
 
-template <bool kFromAmax>
+__device__ __forceinline__ void ld_block32(const __nv_bfloat16* p, bool vec32, uint32_t (&w)[8]) {
+  if (vec32) {
+    asm volatile("ld.global.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                 : "l"(p));
+  } else {
+    const uint4 a = ld_stream(p), b = ld_stream(p + 8);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  }
+}
+
+template <bool kFromAmax, bool kReverse, bool kVec32>
 __global__ void __launch_bounds__(256) quantize_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
                                                        int64_t cols, int64_t ldx, const float* __restrict__ scale_src,
                                                        uint8_t* __restrict__ codes, int64_t ld_codes,
@@ -116,54 +133,59 @@ __global__ void __launch_bounds__(256) quantize_kernel(const __nv_bfloat16* __re
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   const int64_t gwarp = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int64_t spans = (cols + 255) / 256;
-  const int64_t total = rows * spans;
-  const int64_t blocks_per_row = cols / 16;
+  const int bpr = static_cast<int>(cols / 16);                 // blocks per row
+  const int steps = (bpr + 31) / 32;
+  const int chunks = (steps + kQuantStepsPerTask - 1) / kQuantStepsPerTask;
+  const int64_t total = rows * chunks;
 
-  for (int64_t t0 = gwarp; t0 < total; t0 += nwarps * kQuantUnroll) {
-    uint4 v[kQuantUnroll];
-    int64_t row[kQuantUnroll], col[kQuantUnroll];
+  for (int64_t t = gwarp; t < total; t += nwarps) {
+    const int64_t tt = kReverse ? total - 1 - t : t;
+    const int64_t row = tt / chunks;
+    const int chunk = static_cast<int>(tt - row * chunks);
+    const int st_begin = chunk * kQuantStepsPerTask;
+    const int st_end = min(steps, st_begin + kQuantStepsPerTask);
+    const __nv_bfloat16* xrow = x + row * ldx;
+    uint8_t* crow = codes + row * ld_codes;
+    uint8_t* srow = scales + ((row >> 7) * k_atoms) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4;
+    for (int st = st_begin; st < st_end; st += kQuantUnroll) {
+      uint32_t w[kQuantUnroll][8];
 #pragma unroll
-    for (int u = 0; u < kQuantUnroll; ++u) {
-      const int64_t t = t0 + u * nwarps;
-      row[u] = t / spans;
-      col[u] = (t - row[u] * spans) * 256 + lane * 8;
-      v[u] = make_uint4(0, 0, 0, 0);
-      if (t < total && col[u] < cols) v[u] = ld_stream(x + row[u] * ldx + col[u]);
-    }
+      for (int u = 0; u < kQuantUnroll; ++u) {
+        const int blk = (st + u) * 32 + lane;
 #pragma unroll
-    for (int u = 0; u < kQuantUnroll; ++u) {
-      const int64_t t = t0 + u * nwarps;
-      if (t >= total) break;  // warp-uniform
-      const bool valid = col[u] < cols;
-      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-      float f[8];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        for (int i = 0; i < 8; ++i) w[u][i] = 0;
+        if (st + u < st_end && blk < bpr) ld_block32(xrow + blk * 16, kVec32, w[u]);
       }
-      uint32_t mb = max(max(bf16x2_absmax_bits(w[0]), bf16x2_absmax_bits(w[1])),
-                        max(bf16x2_absmax_bits(w[2]), bf16x2_absmax_bits(w[3])));
-      mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 1));
-      const float amax_b = __uint_as_float(mb << 16);
-      float inv;
-      uint32_t s = block_scale(amax_b, g, inv);
-      float q[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(f[i], inv);
-      uint32_t packed = e2m1x8(q);
-      if (inv == 0.0f) packed = 0;
-      if (!valid) s = 0;
-      if (valid) *reinterpret_cast<uint32_t*>(codes + row[u] * ld_codes + col[u] / 2) = packed;
-      // four consecutive blocks' scales share one aligned 32-bit word of the scale layout
-      const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, s, 2);
-      const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, s, 4);
-      const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, s, 6);
-      const int64_t blk = col[u] / 16;
-      if ((lane & 7) == 0 && blk < blocks_per_row) {
-        *reinterpret_cast<uint32_t*>(scales + scale_offset(row[u], blk, k_atoms)) =
-            s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      for (int u = 0; u < kQuantUnroll; ++u) {
+        if (st + u >= st_end) break;  // warp-uniform
+        const int blk = (st + u) * 32 + lane;
+        const bool valid = blk < bpr;
+        uint32_t m2 = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m2 = __vmaxu2(m2, w[u][i] & 0x7FFF7FFFu);
+        const uint32_t mb = max(m2 & 0xFFFFu, m2 >> 16);
+        float inv;
+        uint32_t sc = block_scale(__uint_as_float(mb << 16), g, inv);
+        uint32_t packed[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float q[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            q[2 * i] = __fmul_rn(__uint_as_float(w[u][4 * h + i] << 16), inv);
+            q[2 * i + 1] = __fmul_rn(__uint_as_float(w[u][4 * h + i] & 0xFFFF0000u), inv);
+          }
+          packed[h] = (inv == 0.0f) ? 0u : e2m1x8(q);
+        }
+        if (!valid) sc = 0;
+        if (valid) *reinterpret_cast<uint2*>(crow + static_cast<int64_t>(blk) * 8) = make_uint2(packed[0], packed[1]);
+        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
+        const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
+        const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
+        if ((lane & 3) == 0 && valid)
+          *reinterpret_cast<uint32_t*>(srow + static_cast<int64_t>(blk >> 2) * 512) =
+              sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
       }
     }
   }

@@ -21,7 +21,8 @@
  *
  * Conventions for every entry point:
  *   - All pointers inside the structs and all data pointers are DEVICE pointers, owned by the caller.
- *     The library allocates nothing and frees nothing.
+ *     The library allocates no memory the caller sees; its only allocation is the split-K scratch of
+ *     nvfp4_linear for K >= 32768 (see nvfp4_linear_split_k).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default stream).  Host-side
  *     argument checks run before anything is launched; when one fails nothing is launched and the
  *     status says why.  Nothing throws, prints or traps.
@@ -163,6 +164,13 @@ NVFP4_API nvfp4_status nvfp4_get_device_error(nvfp4_stream_t stream);
 /* Column tile width the GEMM uses for a weight of N rows and K columns and an epilogue kind; it
  * depends on (N, K, kind) only, never on M.  0 when the shape is unsupported. */
 NVFP4_API int32_t nvfp4_linear_tile_n(int64_t N, int64_t K, int32_t kind);
+
+/* Number of K splits the GEMM uses for a weight of N rows and K columns and an epilogue kind: 2 when
+ * K >= 32768 (except the head-norm epilogue), else 1; it depends on (N, K, kind) only, never on M.
+ * A split GEMM keeps per-stream scratch in device memory that the library allocates on first use
+ * (and regrows when a larger problem needs more); make the first such call on a stream outside
+ * stream capture.  0 when the shape is unsupported. */
+NVFP4_API int32_t nvfp4_linear_split_k(int64_t N, int64_t K, int32_t kind);
 
 /* Static string naming a status code. */
 NVFP4_API const char* nvfp4_status_string(nvfp4_status status);

@@ -145,6 +145,29 @@ def test_tile_n_128_path_and_k_tail(lib):
     check(f32(out), ref["y"], "bn128")
 
 
+@pytest.mark.parametrize("kind,M,N", [("bias", 130, 256), ("bias", 257, 384), ("resid_gate", 129, 256),
+                                      ("gated_silu", 131, 512)])
+def test_split_k_long_reduction(lib, kind, M, N):
+    """K >= 32768 runs as two K halves whose fp32 partials are summed before the epilogue."""
+    K = 32768
+    assert B.split_k(N, K, kind) == 2 and B.split_k(N, 4608, kind) == 1 and B.split_k(13824, K, "qknorm") == 1
+    if kind == "bias":
+        case = W.case_bias(M, N, K, seed=M, w_std=0.01, x_dist="student_t")
+    elif kind == "resid_gate":
+        case = W.case_ffn_down(M, N=N, F=K, seed=M)
+    else:
+        case = W.case_ffn_up(M, K=K, F=N // 2, seed=M)
+    aq, wq, out = run_gpu(case)
+    _, _, ref = run_oracle(case)
+    check(f32(out), ref["y"], f"split-K {kind}")
+    # which K half finishes first varies from run to run; the result may not
+    bias = case.bias.cuda() if case.bias is not None else None
+    for _ in range(3):
+        again = B.linear(aq, wq, case.epilogue, bias=bias, **gpu_epi_kwargs(case))
+        B.check_device_error()
+        assert torch.equal(again, out)
+
+
 # ------------------------------------------------------------------------------------------
 # row independence (bitwise, on the GPU)
 # ------------------------------------------------------------------------------------------
