@@ -19,9 +19,9 @@ LIB_PATH = os.path.join(_HERE, "libnvfp4.so")
 #: every function the header declares
 EXPORTS = ("nvfp4_quantize", "nvfp4_linear", "nvfp4_dequantize", "nvfp4_amax", "nvfp4_scale_bytes",
            "nvfp4_scale_offset", "nvfp4_get_device_error", "nvfp4_linear_tile_n", "nvfp4_linear_split_k",
-           "nvfp4_status_string", "nvfp4_version")
+           "nvfp4_status_string", "nvfp4_version", "nvfp4_linear_noalloc", "nvfp4_linear_noalloc_scratch_bytes")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_MISALIGNED, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_MISALIGNED, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_SCRATCH_LIMIT = range(7)
 EPI_BIAS, EPI_QKNORM, EPI_GATED_SILU, EPI_RESID_GATE = range(4)
 EPI_KINDS = {"bias": EPI_BIAS, "qknorm": EPI_QKNORM, "gated_silu": EPI_GATED_SILU, "resid_gate": EPI_RESID_GATE}
 
@@ -62,6 +62,8 @@ def load() -> ctypes.CDLL:
     sig = {
         "nvfp4_quantize": (I32, [P, I64, I64, I64, I32, TP, P]),
         "nvfp4_linear": (I32, [TP, TP, EP, P, I64, TP, P]),
+        "nvfp4_linear_noalloc": (I32, [TP, TP, EP, P, I64, TP, P]),
+        "nvfp4_linear_noalloc_scratch_bytes": (SZ, []),
         "nvfp4_dequantize": (I32, [TP, P, I64, P]),
         "nvfp4_amax": (I32, [P, I64, I64, I64, P, P]),
         "nvfp4_scale_bytes": (SZ, [I64, I64]),

@@ -31,6 +31,27 @@ struct DeviceState {
 std::mutex g_mutex;
 DeviceState g_devices[kMaxDevices];
 
+// Fixed split-K scratch for nvfp4_linear_noalloc: a file-scope device array, so that entry point
+// never allocates.  Every device that loads the library holds it until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once per device.  In host
+// code the array's name is only a host-side handle, so kernels must be given this address.
+nvfp4_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_noalloc_scratch_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return NVFP4_ERR_CUDA;
+    g_noalloc_scratch_addr[dev] = ptr;
+  }
+  *out = g_noalloc_scratch_addr[dev];
+  return NVFP4_OK;
+}
+
 // Split-K scratch, one buffer per (device, stream) so that calls on different streams never share
 // it.  Grown on demand; growing frees the old buffer (cudaFree waits for the device).
 struct Scratch {
@@ -191,6 +212,7 @@ const char* nvfp4_status_string(nvfp4_status s) {
     case NVFP4_ERR_MISALIGNED: return "misaligned pointer or leading dimension";
     case NVFP4_ERR_CUDA: return "CUDA runtime error";
     case NVFP4_ERR_DEVICE_TIMEOUT: return "device-side pipeline wait timed out";
+    case NVFP4_ERR_SCRATCH_LIMIT: return "split-K scratch needed exceeds the fixed buffer of nvfp4_linear_noalloc";
   }
   return "unknown status";
 }
@@ -273,8 +295,15 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor* t, void* out_bf16, int64_t ld_
   return launch_status();
 }
 
-nvfp4_status nvfp4_linear(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvfp4_epilogue_desc* epi,
-                          void* out_bf16, int64_t ld_out, const nvfp4_tensor* out_fp4, nvfp4_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The fused linear; `fixed_scratch` selects the split-K scratch: the library's per-stream buffer
+// (nvfp4_linear) or the fixed file-scope array (nvfp4_linear_noalloc).
+nvfp4_status linear_impl(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvfp4_epilogue_desc* epi,
+                         void* out_bf16, int64_t ld_out, const nvfp4_tensor* out_fp4, nvfp4_stream_t stream,
+                         bool fixed_scratch) {
   if (!epi) return NVFP4_ERR_INVALID_ARG;
   if (nvfp4_status e = check_tensor(a, true, 16)) return e;
   if (nvfp4_status e = check_tensor(w, true, 16)) return e;
@@ -358,7 +387,12 @@ nvfp4_status nvfp4_linear(const nvfp4_tensor* a, const nvfp4_tensor* w, const nv
     const size_t flag_bytes = (static_cast<size_t>(g.num_tiles) * 4 + 255) & ~size_t(255);
     const size_t part_bytes = static_cast<size_t>(g.num_tiles) * 2 * 128 * cols_per_thread * 4;
     void* ws = nullptr;
-    if (nvfp4_status e = scratch_for(s, flag_bytes + part_bytes, &ws)) return e;
+    if (fixed_scratch) {
+      if (flag_bytes + part_bytes > kNoAllocScratchBytes) return NVFP4_ERR_SCRATCH_LIMIT;
+      if (nvfp4_status e = noalloc_scratch(&ws)) return e;
+    } else if (nvfp4_status e = scratch_for(s, flag_bytes + part_bytes, &ws)) {
+      return e;
+    }
     g.split_flags = static_cast<unsigned int*>(ws);
     g.split_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + flag_bytes);
     if (cudaMemsetAsync(ws, 0, static_cast<size_t>(g.num_tiles) * 4, s) != cudaSuccess) return NVFP4_ERR_CUDA;
@@ -374,6 +408,28 @@ nvfp4_status nvfp4_linear(const nvfp4_tensor* a, const nvfp4_tensor* w, const nv
   }
   return NVFP4_ERR_INVALID_ARG;
 }
+
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_linear(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvfp4_epilogue_desc* epi,
+                          void* out_bf16, int64_t ld_out, const nvfp4_tensor* out_fp4, nvfp4_stream_t stream) {
+  return linear_impl(a, w, epi, out_bf16, ld_out, out_fp4, stream, false);
+}
+
+// Same computation as nvfp4_linear, for callers that must not allocate device memory: the split-K
+// scratch of long-K calls lives in a fixed 64 MiB device array instead of a buffer the library
+// allocates.  The array's address is looked up on the first call on each device.  Calls whose
+// scratch would not fit return NVFP4_ERR_SCRATCH_LIMIT before launching anything.  All calls on a
+// device share the array, so calls that overlap on the GPU race.
+nvfp4_status nvfp4_linear_noalloc(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvfp4_epilogue_desc* epi,
+                                  void* out_bf16, int64_t ld_out, const nvfp4_tensor* out_fp4,
+                                  nvfp4_stream_t stream) {
+  return linear_impl(a, w, epi, out_bf16, ld_out, out_fp4, stream, true);
+}
+
+size_t nvfp4_linear_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 nvfp4_status nvfp4_get_device_error(nvfp4_stream_t stream) {
   DeviceState* st;

@@ -54,7 +54,9 @@ typedef enum {
   NVFP4_ERR_UNSUPPORTED_SHAPE = 2, /* a size rule below is not met                                   */
   NVFP4_ERR_MISALIGNED = 3,        /* a pointer or leading dimension is not 16-byte aligned           */
   NVFP4_ERR_CUDA = 4,              /* a CUDA runtime call failed                                      */
-  NVFP4_ERR_DEVICE_TIMEOUT = 5     /* a kernel's pipeline wait ran out of time and the kernel gave up */
+  NVFP4_ERR_DEVICE_TIMEOUT = 5,    /* a kernel's pipeline wait ran out of time and the kernel gave up */
+  NVFP4_ERR_SCRATCH_LIMIT = 6      /* nvfp4_linear_noalloc: the problem needs more split-K scratch than
+                                      its fixed buffer holds                                          */
 } nvfp4_status;
 
 /*
@@ -140,6 +142,32 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols,
  */
 NVFP4_API nvfp4_status nvfp4_linear(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvfp4_epilogue_desc* epi,
                           void* out_bf16, int64_t ld_out, const nvfp4_tensor* out_fp4, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_linear for callers that cannot allocate device memory.  The paper has no counterpart to this
+ * entry point; it exists for how the library is called, not for what it computes.  Some callers must not call cudaMalloc from inside this library: code that
+ * runs while a serving runtime or framework owns all device memory through its own pool, code on a
+ * latency-critical path where cudaMalloc / cudaFree would synchronise the device, and code that records
+ * work for later replay.  This entry point computes exactly what nvfp4_linear computes, with the same
+ * arguments and rules, but the split-K scratch of long-K calls (K >= 32768, see nvfp4_linear_split_k)
+ * lives in a fixed device array of nvfp4_linear_noalloc_scratch_bytes() bytes (64 MiB) built into the
+ * library instead of a buffer it allocates; calls without split-K need no scratch at all.
+ *   - It calls no cudaMalloc, cudaFree or allocating routine.  The array is part of the library's
+ *     device image: every GPU that loads the library holds it until the process exits.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with that
+ *     device current; make that first call before any stream capture.
+ *   - A call whose scratch would not fit returns NVFP4_ERR_SCRATCH_LIMIT and launches nothing.  The
+ *     scratch of a split-K call is 4 bytes per output tile plus 128 KiB per 128 x 256 tile.
+ *   - All calls on a device share the one array, which keeps the previous call's contents; each call
+ *     clears the part that must start at zero.  Calls that overlap on the GPU (different streams without
+ *     ordering between them) race on the array and give wrong results: order them.
+ */
+NVFP4_API nvfp4_status nvfp4_linear_noalloc(const nvfp4_tensor* a, const nvfp4_tensor* w,
+                                            const nvfp4_epilogue_desc* epi, void* out_bf16, int64_t ld_out,
+                                            const nvfp4_tensor* out_fp4, nvfp4_stream_t stream);
+
+/* Size in bytes of the fixed split-K scratch array used by nvfp4_linear_noalloc. */
+NVFP4_API size_t nvfp4_linear_noalloc_scratch_bytes(void);
 
 /* Dequantise t to bf16 [t->rows, ld_out]: value = e2m1(code) * (e4m3(scale) * g), each product in fp32
  * rounded to nearest even, then rounded to bf16.  Rules as for nvfp4_quantize. */
