@@ -16,9 +16,9 @@
 //                 accumulator row 32q+i (TMEM lane = row) and half of the tile's columns.  It copies its
 //                 columns into registers, releases TMEM at once (`acc_empty`) so the next tile's MMAs
 //                 start, then applies bias / head RMSNorm / gated SiLU / residual+gate and the NVFP4
-//                 requantisation from registers.  Row-wise reductions are thread-local: the 256-wide
-//                 head's sum of squares reads the other half straight from TMEM before the release, so
-//                 there is no cross-fragment exchange and no revisit of the output.
+//                 requantisation from registers.  Row-wise reductions stay within the two threads that
+//                 hold a row: for the 256-wide head each adds the squares of its 128 columns and the
+//                 two partial sums meet in shared memory, so the head is never revisited.
 //                 Stores go through a 1 KB per-warp shared-memory transpose so that each st.global
 //                 writes whole 32-byte row segments.
 // The per-stage TMEM scale slot is safe to rewrite without extra waits: the producer refills stage s
@@ -33,6 +33,14 @@ namespace nvfp4 {
 enum EpiKind : int { kEpiBias = 0, kEpiQkNorm = 1, kEpiGatedSilu = 2, kEpiResidGate = 3 };
 
 enum DeviceError : unsigned int { kErrNone = 0, kErrTimeout = 5 };
+
+// MMAs of K = 64 per pipeline stage: 2 (64-byte rows, 64-byte swizzle) or 4 (128-byte rows).
+#ifndef NVFP4_STAGE_KSTEPS
+#define NVFP4_STAGE_KSTEPS 4
+#endif
+constexpr int kStageKSteps = NVFP4_STAGE_KSTEPS;
+constexpr int kStageRowBytes = 32 * kStageKSteps;  // code bytes of one row per stage
+static_assert(kStageKSteps == 2 || kStageKSteps == 4, "stage depth");
 
 struct GemmArgs {
   int32_t M, N, K;
@@ -87,14 +95,14 @@ template <int BN>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int THREADS = 512;
-  static constexpr int BK_BYTES = 128;                  // 256 E2M1 elements per stage and row
-  static constexpr int KSTEPS = 4;                      // MMAs of K = 64 per stage
+  static constexpr int KSTEPS = kStageKSteps;           // MMAs of K = 64 per stage
+  static constexpr int BK_BYTES = kStageRowBytes;       // 64 * KSTEPS E2M1 elements per stage and row
   static constexpr int A_BYTES = BM * BK_BYTES;
   static constexpr int B_BYTES = BN * BK_BYTES;
-  static constexpr int SFA_BYTES = 4 * 512;             // 128 rows x 16 blocks
-  static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;
+  static constexpr int SF_ATOM_BYTES = 512;             // 128 rows x 4 blocks
+  static constexpr int SFA_BYTES = KSTEPS * SF_ATOM_BYTES;
+  static constexpr int SFB_BYTES = (BN / 128) * KSTEPS * SF_ATOM_BYTES;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
   static constexpr int ACC_BUFS = BN == 256 ? 1 : 2;
   static constexpr int SF_COL0 = ACC_BUFS * BN;         // TMEM columns after the accumulator(s)
   static constexpr int SFA_COLS = KSTEPS * 4;
@@ -103,13 +111,20 @@ struct GemmCfg {
   static constexpr int TMEM_COLS = 512;
   static constexpr int EPI_WARPS = 8;
   static constexpr int XPOSE_BYTES = 1024;              // per epilogue warp: 32 rows x 32 bytes
-  static constexpr int AUX_BYTES = 512;                 // barriers and flags
+  static constexpr int AUX_BYTES = 1536;                // barriers, flags, head-norm partial sums
+  static constexpr int SS_OFFSET = 512;                 // float [2][128] partial sums of squares
+  static constexpr int SMEM_LIMIT = 232448;
+  // as many stages as shared memory and the TMEM scale slots allow
+  static constexpr int STAGES_SMEM = (SMEM_LIMIT - AUX_BYTES - 1023 - EPI_WARPS * XPOSE_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES_TMEM = (TMEM_COLS - SF_COL0) / SF_COLS;
+  static constexpr int STAGES = STAGES_SMEM < STAGES_TMEM ? STAGES_SMEM : STAGES_TMEM;
   static constexpr int SMEM_BYTES = AUX_BYTES + 1023 + STAGES * STAGE_BYTES + EPI_WARPS * XPOSE_BYTES;
   static constexpr uint32_t IDESC = idesc_nvf4(BM, BN);
   static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");
-  static_assert(SF_COLS % 16 == 0, "scale slot is written 16 columns at a time");
-  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert((4 * STAGES + 5) * 8 + 16 <= AUX_BYTES, "barrier area");
+  static_assert(SF_COLS % 8 == 0, "scale slot is written 8 columns at a time");
+  static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
+  static_assert(STAGE_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
+  static_assert((4 * STAGES + 5) * 8 + 16 <= SS_OFFSET, "barrier area");
   static_assert(BM == 128, "the split-K partial layout assumes 128 rows per tile");
 };
 
@@ -228,10 +243,9 @@ template <int BN, int KIND>
 struct Epilogue {
   static constexpr int COLS = (KIND == kEpiGatedSilu) ? 128 : BN / 2;  // accumulator columns per thread
 
-  // Copy this thread's accumulator columns into `acc`; for the head RMSNorm also return the sum of
-  // squares of the whole biased 256-wide row (the other half is read from TMEM and dropped).
-  static __device__ __forceinline__ void load(const GemmArgs& a, uint32_t t_acc, int e, int nb, float alpha,
-                                              bool norm, float* acc, float& ss) {
+  // Copy this thread's accumulator columns into `acc` (gated SiLU: its 64 a columns, then the 64
+  // matching b columns).
+  static __device__ __forceinline__ void load(uint32_t t_acc, int e, float* acc) {
     if constexpr (KIND == kEpiGatedSilu) {
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -241,35 +255,30 @@ struct Epilogue {
     } else {
 #pragma unroll
       for (int c = 0; c < COLS / 32; ++c) tmem_load32(t_acc + COLS * e + 32 * c, acc + 32 * c);
-      if constexpr (KIND == kEpiQkNorm) {
-        ss = 0.0f;
-        if (norm) {
-          const int col_base = nb * BN;
+    }
+  }
+
+  // Sum of squares of the biased 256-wide head of this row: each of the row's two threads adds its
+  // 128 columns, and the partial sums meet in shared memory (both epilogue warpgroups take part).
+  static __device__ __forceinline__ float head_sumsq(const GemmArgs& a, int e, int nb, int row_local, float alpha,
+                                                     const float* acc, float* ss_x) {
+    float ss = 0.0f;
+    const int col_e = nb * BN + COLS * e;
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
+    for (int g = 0; g < COLS / 16; ++g) {
+      float b[16];
+      if (a.bias != nullptr) load_bf16x16(a.bias + col_e + 16 * g, b);
 #pragma unroll
-            for (int g = 0; g < COLS / 16; ++g) {
-              float other[16];
-              if (half != e) {
-                uint32_t r[16];
-                tmem_ld_32x32b_x16(t_acc + COLS * half + 16 * g, r);
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) other[i] = __uint_as_float(r[i]);
-              }
-              float b[16];
-              if (a.bias != nullptr) load_bf16x16(a.bias + col_base + COLS * half + 16 * g, b);
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float raw = (half != e) ? other[i] : acc[16 * g + i];
-                const float v = raw * alpha + (a.bias != nullptr ? b[i] : 0.0f);
-                ss = fmaf(v, v, ss);
-              }
-            }
-          }
-        }
+      for (int i = 0; i < 16; ++i) {
+        const float v = acc[16 * g + i] * alpha + (a.bias != nullptr ? b[i] : 0.0f);
+        ss = fmaf(v, v, ss);
       }
     }
+    ss_x[e * 128 + row_local] = ss;
+    named_barrier_sync(2, 256);
+    ss += ss_x[(1 - e) * 128 + row_local];
+    named_barrier_sync(2, 256);  // the next tile may overwrite the slots only after both reads
+    return ss;
   }
 
   static __device__ __forceinline__ void finish(const GemmArgs& a, uint8_t* xpose, int row0, int row, int e, int nb,
@@ -413,6 +422,7 @@ __global__ void __launch_bounds__(512, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* never_abort = abort_flag + 1;  // stays 0: drains must not be cut short by an abort
   volatile int* split_role = never_abort + 1;
+  float* ss_x = reinterpret_cast<float*>(smem_raw + C::SS_OFFSET);
   uint8_t* ring = smem_raw + C::AUX_BYTES;
   ring += (1024u - (smem_u32(ring) & 1023u)) & 1023u;
   uint8_t* xpose_all = ring + C::STAGES * C::STAGE_BYTES;
@@ -474,13 +484,13 @@ __global__ void __launch_bounds__(512, 1)
             uint8_t* ssfa = sb + C::B_BYTES;
             uint8_t* ssfb = ssfa + C::SFA_BYTES;
             mbar_arrive_expect_tx(&sf_landed[stage], sf_bytes * (1 + BN / 128));
-            bulk_load(ssfa, args.sfa + (static_cast<int64_t>(mb) * args.k_atoms + kb * 4) * 512, sf_bytes,
+            bulk_load(ssfa, args.sfa + (static_cast<int64_t>(mb) * args.k_atoms + kb * C::KSTEPS) * 512, sf_bytes,
                       &sf_landed[stage]);
 #pragma unroll
             for (int j = 0; j < BN / 128; ++j)
-              bulk_load(ssfb + j * 2048,
+              bulk_load(ssfb + j * C::KSTEPS * C::SF_ATOM_BYTES,
                         args.sfb + (static_cast<int64_t>(b_row0<BN, KIND>(args, nb, j) / 128) * args.k_atoms +
-                                    kb * 4) * 512,
+                                    kb * C::KSTEPS) * 512,
                         sf_bytes, &sf_landed[stage]);
             mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES);
             tma_load_2d(sa, &tmap_a, &full[stage], kb * C::BK_BYTES, mb * C::BM);
@@ -534,7 +544,8 @@ __global__ void __launch_bounds__(512, 1)
             const uint32_t sfa_t = tmem_base + C::SF_COL0 + stage * C::SF_COLS;
             const uint32_t sfb_t = sfa_t + C::SFA_COLS;
             for (int k = 0; k < ks; ++k)
-              tc_mma_nvf4(d_tmem, desc_kmajor_sw128(a_addr + k * 32), desc_kmajor_sw128(b_addr + k * 32), C::IDESC,
+              tc_mma_nvf4(d_tmem, desc_kmajor_swizzled<C::BK_BYTES>(a_addr + k * 32),
+                          desc_kmajor_swizzled<C::BK_BYTES>(b_addr + k * 32), C::IDESC,
                           (kb != wu.kb0 || k != 0) ? 1u : 0u, sfa_t + k * 4, sfb_t + k * (BN / 32));
             tc_commit(&empty[stage]);
             if (++stage == C::STAGES) {
@@ -563,6 +574,7 @@ __global__ void __launch_bounds__(512, 1)
     // 4 scales of one K step from column r / 32 of that step's group of 4 columns, identically in
     // every sub-partition; 16-byte row i of a 512-byte scale atom is exactly those 4 columns of lane i.
     const int q = warp & 3;
+    constexpr int NV = C::SF_COLS / 4;  // 16-byte vectors per lane and stage
     int stage = 0;
     uint32_t phase = 0;
     for (int u = blockIdx.x; u < args.num_units; u += gridDim.x) {
@@ -578,32 +590,31 @@ __global__ void __launch_bounds__(512, 1)
         const uint8_t* ssfb = ssfa + C::SFA_BYTES;
         const int ks = min(C::KSTEPS, args.k_steps - kb * C::KSTEPS);
         const uint32_t t_sf = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + C::SF_COL0 + stage * C::SF_COLS;
-        // slot column order: A steps 0..3 (4 columns each), then for each step k the weight's
+        // slot column order: A steps 0..KSTEPS-1 (4 columns each), then for each step k the weight's
         // 128-row blocks j = 0 .. BN/128-1 (4 columns each)
-        constexpr int NV = C::SF_COLS / 4;  // 16-byte vectors per lane
 #pragma unroll
-        for (int grp = 0; grp < NV / 4; ++grp) {
-          uint32_t v[16];
+        for (int grp = 0; grp < NV / 2; ++grp) {
+          uint32_t v[8];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int idx = grp * 4 + u;
+          for (int h = 0; h < 2; ++h) {
+            const int idx = grp * 2 + h;
             int k;
             const uint8_t* src;
-            if (idx < 4) {
+            if (idx < C::KSTEPS) {
               k = idx;
-              src = ssfa + k * 512;
+              src = ssfa + k * C::SF_ATOM_BYTES;
             } else {
-              k = (idx - 4) / (BN / 128);
-              src = ssfb + ((idx - 4) % (BN / 128)) * 2048 + k * 512;
+              k = (idx - C::KSTEPS) / (BN / 128);
+              src = ssfb + ((idx - C::KSTEPS) % (BN / 128)) * C::KSTEPS * C::SF_ATOM_BYTES + k * C::SF_ATOM_BYTES;
             }
             uint4 x = make_uint4(0, 0, 0, 0);
             if (k < ks) x = *reinterpret_cast<const uint4*>(src + lane * 16);
-            v[4 * u + 0] = x.x;
-            v[4 * u + 1] = x.y;
-            v[4 * u + 2] = x.z;
-            v[4 * u + 3] = x.w;
+            v[4 * h + 0] = x.x;
+            v[4 * h + 1] = x.y;
+            v[4 * h + 2] = x.z;
+            v[4 * h + 3] = x.w;
           }
-          tmem_st_32x32b_x16(t_sf + grp * 16, v);
+          tmem_st_32x32b_x8(t_sf + grp * 8, v);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -647,8 +658,7 @@ __global__ void __launch_bounds__(512, 1)
       const int row0 = mb * C::BM + q * 32;
       const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(abuf * BN);
       float acc[E::COLS];
-      float ss = 0.0f;
-      E::load(args, t_acc, e, nb, alpha, gamma != nullptr, acc, ss);
+      E::load(t_acc, e, acc);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[abuf]);
@@ -660,6 +670,8 @@ __global__ void __launch_bounds__(512, 1)
       if (KIND != kEpiQkNorm && args.splits > 1 &&
           !split_exchange<E::COLS>(args, wu.tile, e, q * 32 + lane, acc, split_role, abort_flag))
         continue;
+      float ss = 0.0f;
+      if (KIND == kEpiQkNorm && gamma != nullptr) ss = E::head_sumsq(args, e, nb, q * 32 + lane, alpha, acc, ss_x);
       E::finish(args, xpose, row0, row0 + lane, e, nb, alpha, qg, gamma, ss, acc);
     }
   }

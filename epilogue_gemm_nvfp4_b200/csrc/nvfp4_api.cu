@@ -152,17 +152,19 @@ int resident_grid(Kernel kernel, int threads, int64_t work_items, int items_per_
   return static_cast<int>(g);
 }
 
-// 2-D TMA descriptor over packed E2M1 codes viewed as bytes: [rows][cols/2], box 128 x 128 bytes,
-// 128-byte swizzle (the layout the tensor-core descriptors expect).
+// 2-D TMA descriptor over packed E2M1 codes viewed as bytes: [rows][cols/2], box of 128 rows x one
+// stage's row bytes, swizzled by that width (the layout the tensor-core descriptors expect).
 nvfp4_status make_code_map(CUtensorMap* map, const nvfp4_tensor* t) {
   auto encode = tensor_map_encoder();
   if (!encode) return NVFP4_ERR_CUDA;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(t->cols / 2), static_cast<cuuint64_t>(t->rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_codes_of(t))};
-  cuuint32_t box[2] = {128, 128};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kStageRowBytes), 128};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, t->codes, dims, strides, box, estr,
-                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      kStageRowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

@@ -174,6 +174,13 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// 32 lanes x 8 consecutive 32-bit columns <- 8 registers per thread (thread i writes lane i).
+__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 // 32 lanes x 16 consecutive 32-bit columns <- 16 registers per thread (thread i writes lane i).
 __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
@@ -226,15 +233,19 @@ __device__ __forceinline__ void bulk_wait_group_read() {
 // Wait until every committed bulk group of this thread has completed (writes included).
 __device__ __forceinline__ void bulk_wait_group_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// Shared-memory matrix descriptor, K-major operand written by TMA with the 128-byte swizzle:
-// rows of 128 bytes, 8-row (1024-byte) swizzle atoms stacked densely along M/N.
-__device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
+// Shared-memory matrix descriptor, K-major operand written by TMA with a kRowBytes-byte swizzle
+// (128 or 64): rows of kRowBytes bytes, 8-row swizzle atoms (8 * kRowBytes bytes) stacked densely
+// along M/N.  The leading offset is unused with swizzling; the stride offset steps to the next
+// 8-row group.
+template <int kRowBytes>
+__device__ __forceinline__ uint64_t desc_kmajor_swizzled(uint32_t saddr) {
+  static_assert(kRowBytes == 128 || kRowBytes == 64, "128- or 64-byte swizzle");
   uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);   // start address, 16-byte units
-  d |= static_cast<uint64_t>(1) << 16;                    // leading offset (unused with swizzle)
-  d |= static_cast<uint64_t>(1024 >> 4) << 32;            // stride offset: next 8-row group
-  d |= static_cast<uint64_t>(1) << 46;                    // descriptor version for sm_100
-  d |= static_cast<uint64_t>(2) << 61;                    // layout: 128-byte swizzle
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);             // start address, 16-byte units
+  d |= static_cast<uint64_t>(1) << 16;                              // leading offset (unused)
+  d |= static_cast<uint64_t>((8 * kRowBytes) >> 4) << 32;           // stride offset: next 8-row group
+  d |= static_cast<uint64_t>(1) << 46;                              // descriptor version for sm_100
+  d |= static_cast<uint64_t>(kRowBytes == 128 ? 2 : 4) << 61;       // layout: 128- / 64-byte swizzle
   return d;
 }
 
