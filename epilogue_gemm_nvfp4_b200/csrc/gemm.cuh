@@ -155,9 +155,10 @@ __device__ __forceinline__ void load_bf16x16(const __nv_bfloat16* p, float (&f)[
   }
 }
 
+// Two floats -> two bf16 (round to nearest even) in one 32-bit word, `lo` in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(lo))) |
-         (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
+  const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&p);
 }
 
 __device__ __forceinline__ void tmem_load32(uint32_t taddr, float* v) {
@@ -303,7 +304,7 @@ struct Epilogue {
               ya += ba[i];
               yb += bb[i];
             }
-            o[16 * g + i] = ya / (1.0f + __expf(-ya)) * yb;
+            o[16 * g + i] = __fdividef(ya, 1.0f + __expf(-ya)) * yb;  // silu(a) * b
           }
         }
         emit_row32(a, xpose, row0, row, ocol, o, qg);

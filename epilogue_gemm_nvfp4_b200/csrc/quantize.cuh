@@ -125,7 +125,7 @@ __device__ __forceinline__ void ld_block32(const __nv_bfloat16* p, bool vec32, u
 }
 
 template <bool kFromAmax, bool kReverse, bool kVec32>
-__global__ void __launch_bounds__(256) quantize_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
+__global__ void __launch_bounds__(256, 6) quantize_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
                                                        int64_t cols, int64_t ldx, const float* __restrict__ scale_src,
                                                        uint8_t* __restrict__ codes, int64_t ld_codes,
                                                        uint8_t* __restrict__ scales, int64_t k_atoms) {
@@ -136,14 +136,15 @@ __global__ void __launch_bounds__(256) quantize_kernel(const __nv_bfloat16* __re
   const int bpr = static_cast<int>(cols / 16);                 // blocks per row
   const int steps = (bpr + 31) / 32;
   const int chunks = (steps + kQuantStepsPerTask - 1) / kQuantStepsPerTask;
+  const int per_chunk = (steps + chunks - 1) / chunks;  // equal chunks of at most kQuantStepsPerTask steps
   const int64_t total = rows * chunks;
 
   for (int64_t t = gwarp; t < total; t += nwarps) {
     const int64_t tt = kReverse ? total - 1 - t : t;
     const int64_t row = tt / chunks;
     const int chunk = static_cast<int>(tt - row * chunks);
-    const int st_begin = chunk * kQuantStepsPerTask;
-    const int st_end = min(steps, st_begin + kQuantStepsPerTask);
+    const int st_begin = chunk * per_chunk;
+    const int st_end = min(steps, st_begin + per_chunk);
     const __nv_bfloat16* xrow = x + row * ldx;
     uint8_t* crow = codes + row * ld_codes;
     uint8_t* srow = scales + ((row >> 7) * k_atoms) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4;
