@@ -126,6 +126,7 @@ struct GemmCfg {
   static_assert(STAGE_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
   static_assert((4 * STAGES + 5) * 8 + 16 <= SS_OFFSET, "barrier area");
   static_assert(BM == 128, "the split-K partial layout assumes 128 rows per tile");
+  static_assert((SMEM_LIMIT >> 4) < (1 << 14), "operand descriptors advance by adds inside the 14-bit address field");
 };
 
 __device__ __forceinline__ void raise_device_error(unsigned int* word, unsigned int code, volatile int* abort) {
@@ -519,8 +520,17 @@ __global__ void __launch_bounds__(512, 1)
     } else if (warp == 1) {
       if (lane == 0) {
         // ---------------------------------------------------------------- MMA issuer
+        // The tensor pipe queues only about two MMAs ahead of this thread, so every instruction
+        // spent here between MMAs is lost tensor time: descriptors and TMEM scale addresses are
+        // formed once and advanced by adds, and a full stage issues its MMAs fully unrolled.
+        constexpr uint64_t kStageDesc = C::STAGE_BYTES >> 4;  // descriptor address units per stage
+        const uint64_t a_desc0 = desc_kmajor_swizzled<C::BK_BYTES>(smem_u32(ring));
+        const uint64_t b_desc_off = C::A_BYTES >> 4;
+        const uint32_t sf_col0 = tmem_base + C::SF_COL0;
         int stage = 0;
         uint32_t phase = 0;
+        uint64_t a_desc = a_desc0;
+        uint32_t sfa_t = sf_col0;
         int abuf = 0;
         uint32_t aphase = 0;
         bool ok = true;
@@ -532,6 +542,7 @@ __global__ void __launch_bounds__(512, 1)
           }
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * BN);
+          uint32_t accumulate = 0;
           for (int kb = wu.kb0; kb < wu.kb1; ++kb) {
             if (!mbar_wait(&sf_full[stage], phase, abort_flag, args.timeout_ns) ||
                 !mbar_wait(&full[stage], phase, abort_flag, args.timeout_ns)) {
@@ -539,19 +550,29 @@ __global__ void __launch_bounds__(512, 1)
               break;
             }
             tc_fence_after();
-            const int ks = min(C::KSTEPS, args.k_steps - kb * C::KSTEPS);
-            const uint32_t a_addr = smem_u32(ring + stage * C::STAGE_BYTES);
-            const uint32_t b_addr = a_addr + C::A_BYTES;
-            const uint32_t sfa_t = tmem_base + C::SF_COL0 + stage * C::SF_COLS;
+            const uint64_t b_desc = a_desc + b_desc_off;
             const uint32_t sfb_t = sfa_t + C::SFA_COLS;
-            for (int k = 0; k < ks; ++k)
-              tc_mma_nvf4(d_tmem, desc_kmajor_swizzled<C::BK_BYTES>(a_addr + k * 32),
-                          desc_kmajor_swizzled<C::BK_BYTES>(b_addr + k * 32), C::IDESC,
-                          (kb != wu.kb0 || k != 0) ? 1u : 0u, sfa_t + k * 4, sfb_t + k * (BN / 32));
+            if (kb * C::KSTEPS + C::KSTEPS <= args.k_steps) {
+#pragma unroll
+              for (int k = 0; k < C::KSTEPS; ++k)
+                tc_mma_nvf4(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::IDESC, accumulate | k, sfa_t + k * 4,
+                            sfb_t + k * (BN / 32));
+            } else {
+              const int ks = args.k_steps - kb * C::KSTEPS;  // K tail: 1 .. KSTEPS-1 steps
+              for (int k = 0; k < ks; ++k)
+                tc_mma_nvf4(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::IDESC, accumulate | k, sfa_t + k * 4,
+                            sfb_t + k * (BN / 32));
+            }
+            accumulate = 1;
             tc_commit(&empty[stage]);
             if (++stage == C::STAGES) {
               stage = 0;
               phase ^= 1u;
+              a_desc = a_desc0;
+              sfa_t = sf_col0;
+            } else {
+              a_desc += kStageDesc;
+              sfa_t += C::SF_COLS;
             }
           }
           if (!ok) break;
