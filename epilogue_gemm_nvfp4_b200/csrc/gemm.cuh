@@ -2,16 +2,19 @@
 //
 // One persistent CTA per SM walks output tiles of 128 rows x BN weight rows (512 threads):
 //   warp 0        TMA producer: per stage, first the scale atoms (bulk copies, counted on `sf_landed`),
-//                 then the A/B code tiles (TMA, 128-byte swizzle, counted on `full`), into a ring of
-//                 shared-memory stages.
+//                 then the A/B code tiles (TMA, 128-byte swizzle, bytes counted on `full`), into a ring
+//                 of shared-memory stages.
 //   warp 1        MMA issuer (one thread): four tcgen05.mma.kind::mxf4nvf4 (K = 64 each) per stage,
 //                 accumulating in TMEM; tcgen05.commit frees the stage (`empty`) and, after the last
 //                 K step of a tile, hands the accumulator to the epilogue (`acc_full`).
 //   warp 2        TMEM allocation / release.
 //   warps 4..7    scale stagers: move each stage's scale atoms from shared memory into that stage's
 //                 TMEM scale slot with tcgen05.st (replicated into the four 32-lane sub-partitions the
-//                 MMA reads), then arrive on `sf_full`.  This keeps scale traffic off the tensor pipe,
-//                 and since the atoms land before the code tiles it overlaps their copy.
+//                 MMA reads), then arrive on the stage's `full` barrier too, so that the MMA thread
+//                 waits once per stage: that thread issues an MMA only every ~128 cycles and spends
+//                 about 100 of them issuing it, so a second wait per stage would idle the tensor pipe.
+//                 This keeps scale traffic off the tensor pipe, and since the atoms land before the
+//                 code tiles it overlaps their copy.
 //   warps 8..15   epilogue, two warpgroups over the same 128 rows: thread i of warp 8+4e+q owns
 //                 accumulator row 32q+i (TMEM lane = row) and half of the tile's columns.  It copies its
 //                 columns into registers, releases TMEM at once (`acc_empty`) so the next tile's MMAs
@@ -124,7 +127,7 @@ struct GemmCfg {
   static_assert(SF_COLS % 8 == 0, "scale slot is written 8 columns at a time");
   static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
   static_assert(STAGE_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
-  static_assert((4 * STAGES + 5) * 8 + 16 <= SS_OFFSET, "barrier area");
+  static_assert((3 * STAGES + 5) * 8 + 16 <= SS_OFFSET, "barrier area");
   static_assert(BM == 128, "the split-K partial layout assumes 128 rows per tile");
   static_assert((SMEM_LIMIT >> 4) < (1 << 14), "operand descriptors advance by adds inside the 14-bit address field");
 };
@@ -170,70 +173,94 @@ __device__ __forceinline__ void tmem_load32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Write 16 bf16 values of this lane's row at column col0 through the warp's transpose buffer: each
-// lane puts its 32-byte row segment into shared memory, then lane pairs store whole segments of
-// 16 rows per st.global.  Rows at or past M are skipped.
-__device__ __forceinline__ void store_row16_bf16(const GemmArgs& a, uint8_t* xpose, int row0, int col0,
+// TMA store maps of the outputs (built on the host; a map is all zeros when its output is absent):
+//   out      bf16 [M][ld_out], box 16 columns x 32 rows, 32-byte swizzle
+//   q_codes  E2M1 bytes [M][ld_q_codes], box 16 bytes x 32 rows, no swizzle
+// The epilogue writes each 32-row block into its warp's 1 KB shared-memory buffer and one lane hands
+// it to the TMA engine: row segments 9 KB apart would otherwise cost the load/store unit one line
+// transaction each, and that unit also carries the MMA thread's barrier traffic.  The map's row count
+// is M, so the engine drops rows at or past M.
+struct OutMaps {
+  CUtensorMap out;
+  CUtensorMap q_codes;
+};
+
+// Wait until the TMA engine has read this warp's buffer (the previous store from it), so that it can
+// be rewritten.  Lane 0 issues all of the warp's bulk stores.
+__device__ __forceinline__ void xpose_acquire() {
+  if ((threadIdx.x & 31) == 0) bulk_wait_group_read<0>();
+  __syncwarp();
+}
+
+// Hand the warp's buffer to the TMA engine as the box at (x, y) of `map`.
+__device__ __forceinline__ void xpose_release(const CUtensorMap* map, const uint8_t* xpose, int x, int y) {
+  fence_proxy_async_smem();  // this thread's shared-memory writes become visible to the TMA engine
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) {
+    tma_store_2d(map, xpose, x, y);
+    bulk_commit_group();
+  }
+}
+
+// Store 16 bf16 values of this lane's row at column col0: lane i writes row i of the 32 x 32-byte box
+// in the 32-byte swizzle (the two 16-byte halves swap every 4 rows, which also keeps the shared-memory
+// writes free of bank conflicts), then the box goes out with one TMA store.
+__device__ __forceinline__ void store_row16_bf16(const OutMaps* om, uint8_t* xpose, int row0, int col0,
                                                  const uint32_t* w) {
   const int lane = threadIdx.x & 31;
-  const int sw = (lane >> 2) & 1;  // the two 16-byte halves swap every 4 rows: no bank conflicts
+  const int sw = (lane >> 2) & 1;
+  xpose_acquire();
   uint4* mine = reinterpret_cast<uint4*>(xpose + lane * 32);
   mine[sw] = make_uint4(w[0], w[1], w[2], w[3]);
   mine[sw ^ 1] = make_uint4(w[4], w[5], w[6], w[7]);
-  __syncwarp();
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int r = 16 * i + (lane >> 1), c = lane & 1;
-    const uint4 v = *reinterpret_cast<const uint4*>(xpose + r * 32 + ((c ^ ((r >> 2) & 1)) * 16));
-    if (row0 + r < a.M)
-      *reinterpret_cast<uint4*>(a.out + static_cast<int64_t>(row0 + r) * a.ld_out + col0 + c * 8) = v;
-  }
-  __syncwarp();
+  xpose_release(&om->out, xpose, col0, row0);
 }
 
 // 32 consecutive output values of one row: bf16 (RNE) output and, when requested, the NVFP4
 // re-quantisation of those bf16 values with the caller's tensor scale (the quantiser's block rule).
-__device__ __forceinline__ void emit_row32(const GemmArgs& a, uint8_t* xpose, int row0, int row, int col0,
-                                           const float* o, float qg) {
+__device__ __forceinline__ void emit_row32(const GemmArgs& a, const OutMaps* om, uint8_t* xpose, int row0, int row,
+                                           int col0, const float* o, float qg) {
   uint32_t packed[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(o[2 * i], o[2 * i + 1]);
   if (a.out != nullptr) {
-    store_row16_bf16(a, xpose, row0, col0, packed);
-    store_row16_bf16(a, xpose, row0, col0 + 16, packed + 8);
+    store_row16_bf16(om, xpose, row0, col0, packed);
+    store_row16_bf16(om, xpose, row0, col0 + 16, packed + 8);
   }
   if (a.q_codes != nullptr) {
-    const int64_t soff = scale_offset(row, col0 / 16, a.q_k_atoms);
-    if (row >= a.M) {
-      *reinterpret_cast<uint16_t*>(a.q_scales + soff) = 0;  // padding rows of the scale layout
-      return;
-    }
-    uint32_t words[4];
-    uint32_t sc[2];
+    // codes and scales of this row's two 16-blocks; rows at or past M get zero scales (the padding
+    // rows of the scale layout) and zero codes, which the TMA store drops
+    uint32_t words[4] = {0u, 0u, 0u, 0u};
+    uint32_t sc[2] = {0u, 0u};
+    if (row < a.M) {
 #pragma unroll
-    for (int blk = 0; blk < 2; ++blk) {
-      float f[16];
-      uint32_t mb = 0;
+      for (int blk = 0; blk < 2; ++blk) {
+        float f[16];
+        uint32_t mb = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint32_t w = packed[8 * blk + i];
-        f[2 * i] = __uint_as_float(w << 16);
-        f[2 * i + 1] = __uint_as_float(w & 0xFFFF0000u);
-        mb = max(mb, bf16x2_absmax_bits(w));
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t w = packed[8 * blk + i];
+          f[2 * i] = __uint_as_float(w << 16);
+          f[2 * i + 1] = __uint_as_float(w & 0xFFFF0000u);
+          mb = max(mb, bf16x2_absmax_bits(w));
+        }
+        float inv;
+        sc[blk] = block_scale(__uint_as_float(mb << 16), qg, inv);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float q[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(f[8 * h + i], inv);
+          words[2 * blk + h] = (inv == 0.0f) ? 0u : e2m1x8(q);
+        }
       }
-      float inv;
-      sc[blk] = block_scale(__uint_as_float(mb << 16), qg, inv);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float q[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(f[8 * h + i], inv);
-        words[2 * blk + h] = (inv == 0.0f) ? 0u : e2m1x8(q);
-      }
     }
-    *reinterpret_cast<uint4*>(a.q_codes + static_cast<int64_t>(row) * a.ld_q_codes + col0 / 2) =
-        make_uint4(words[0], words[1], words[2], words[3]);
-    *reinterpret_cast<uint16_t*>(a.q_scales + soff) = static_cast<uint16_t>(sc[0] | (sc[1] << 8));
+    const int lane = threadIdx.x & 31;
+    xpose_acquire();
+    *reinterpret_cast<uint4*>(xpose + lane * 16) = make_uint4(words[0], words[1], words[2], words[3]);
+    xpose_release(&om->q_codes, xpose, col0 / 2, row0);
+    *reinterpret_cast<uint16_t*>(a.q_scales + scale_offset(row, col0 / 16, a.q_k_atoms)) =
+        static_cast<uint16_t>(sc[0] | (sc[1] << 8));
   }
 }
 
@@ -283,7 +310,8 @@ struct Epilogue {
     return ss;
   }
 
-  static __device__ __forceinline__ void finish(const GemmArgs& a, uint8_t* xpose, int row0, int row, int e, int nb,
+  static __device__ __forceinline__ void finish(const GemmArgs& a, const OutMaps* om, uint8_t* xpose, int row0, int row,
+                                                int e, int nb,
                                                 float alpha, float qg, const __nv_bfloat16* gamma, float ss,
                                                 float* acc) {
     if constexpr (KIND == kEpiGatedSilu) {
@@ -308,7 +336,7 @@ struct Epilogue {
             o[16 * g + i] = __fdividef(ya, 1.0f + __expf(-ya)) * yb;  // silu(a) * b
           }
         }
-        emit_row32(a, xpose, row0, row, ocol, o, qg);
+        emit_row32(a, om, xpose, row0, row, ocol, o, qg);
       }
     } else {
       const int col_e = nb * BN + COLS * e;
@@ -349,7 +377,7 @@ struct Epilogue {
             }
           }
         }
-        emit_row32(a, xpose, row0, row, col0, y, qg);
+        emit_row32(a, om, xpose, row0, row, col0, y, qg);
       }
     }
   }
@@ -408,15 +436,14 @@ __device__ __forceinline__ bool split_exchange(const GemmArgs& a, int tile, int 
 template <int BN, int KIND>
 __global__ void __launch_bounds__(512, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                      const __grid_constant__ GemmArgs args) {
+                      const __grid_constant__ OutMaps out_maps, const __grid_constant__ GemmArgs args) {
   using C = GemmCfg<BN>;
   using E = Epilogue<BN, KIND>;
   extern __shared__ uint8_t smem_raw[];
   // small state first, then the 1024-aligned stage ring (128-byte swizzle atoms), then the transposes
   uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* sf_full = empty + C::STAGES;
-  uint64_t* sf_landed = sf_full + C::STAGES;
+  uint64_t* sf_landed = empty + C::STAGES;
   uint64_t* acc_full = sf_landed + C::STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
@@ -434,9 +461,8 @@ __global__ void __launch_bounds__(512, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 1 + 4);  // the producer's expect-tx arrival + one per scale-stager warp
       mbar_init(&empty[s], 1);
-      mbar_init(&sf_full[s], 4);
       mbar_init(&sf_landed[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -451,6 +477,8 @@ __global__ void __launch_bounds__(512, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmap_a);
     prefetch_tensormap(&tmap_b);
+    if (args.out != nullptr) prefetch_tensormap(&out_maps.out);
+    if (args.q_codes != nullptr) prefetch_tensormap(&out_maps.q_codes);
   }
   if (warp == 2) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -510,6 +538,8 @@ __global__ void __launch_bounds__(512, 1)
         }
         if (!ok) raise_device_error(args.error_word, kErrTimeout, abort_flag);
         // every copy this thread started must land before the CTA's shared memory is released
+        // (`full` also counts the stagers' arrivals: if they stopped on an error, this wait ends at
+        // its time limit instead)
         for (int s = 0; s < C::STAGES; ++s)
           if (armed_mask & (1u << s)) {
             mbar_wait(&sf_landed[s], (armed_parity >> s) & 1u, never_abort, args.timeout_ns);
@@ -544,8 +574,7 @@ __global__ void __launch_bounds__(512, 1)
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * BN);
           uint32_t accumulate = 0;
           for (int kb = wu.kb0; kb < wu.kb1; ++kb) {
-            if (!mbar_wait(&sf_full[stage], phase, abort_flag, args.timeout_ns) ||
-                !mbar_wait(&full[stage], phase, abort_flag, args.timeout_ns)) {
+            if (!mbar_wait(&full[stage], phase, abort_flag, args.timeout_ns)) {
               ok = false;
               break;
             }
@@ -641,7 +670,7 @@ __global__ void __launch_bounds__(512, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sf_full[stage]);
+        if (lane == 0) mbar_arrive(&full[stage]);
         if (++stage == C::STAGES) {
           stage = 0;
           phase ^= 1u;
@@ -694,8 +723,12 @@ __global__ void __launch_bounds__(512, 1)
         continue;
       float ss = 0.0f;
       if (KIND == kEpiQkNorm && gamma != nullptr) ss = E::head_sumsq(args, e, nb, q * 32 + lane, alpha, acc, ss_x);
-      E::finish(args, xpose, row0, row0 + lane, e, nb, alpha, qg, gamma, ss, acc);
+      E::finish(args, &out_maps, xpose, row0, row0 + lane, e, nb, alpha, qg, gamma, ss, acc);
     }
+    // the TMA stores read this warp's buffer and write the outputs asynchronously: both must be done
+    // before the CTA's shared memory is released
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
   }
 
   tc_fence_before();

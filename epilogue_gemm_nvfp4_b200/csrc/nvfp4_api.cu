@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstdlib>
+#include <cstring>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -169,6 +170,36 @@ nvfp4_status make_code_map(CUtensorMap* map, const nvfp4_tensor* t) {
   return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+// TMA store maps of the fused linear's outputs, in the boxes the epilogue writes (32 rows of one warp):
+// bf16 output 16 columns wide with the 32-byte swizzle of its shared-memory buffer, E2M1 codes 16
+// bytes wide unswizzled.  A map stays zeroed when its output is not requested (the kernel never uses it).
+nvfp4_status make_store_maps(OutMaps* om, void* out_bf16, int64_t ld_out, const nvfp4_tensor* out_fp4, int64_t M,
+                             int64_t n_out) {
+  std::memset(om, 0, sizeof(*om));
+  auto encode = tensor_map_encoder();
+  if (!encode) return NVFP4_ERR_CUDA;
+  cuuint32_t estr[2] = {1, 1};
+  if (out_bf16) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(n_out), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_out * 2)};
+    cuuint32_t box[2] = {16, 32};
+    if (encode(&om->out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out_bf16, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return NVFP4_ERR_CUDA;
+  }
+  if (out_fp4) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(n_out / 2), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_codes_of(out_fp4))};
+    cuuint32_t box[2] = {16, 32};
+    if (encode(&om->q_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, out_fp4->codes, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return NVFP4_ERR_CUDA;
+  }
+  return NVFP4_OK;
+}
+
 // Two-way split of K for long reductions (the 53248-wide text projection): a function of K and the
 // epilogue only, never of M, so every row's arithmetic is the same whatever M is.  The head norm takes
 // its sum of squares while loading the accumulator and is never split.
@@ -185,8 +216,8 @@ int tile_n_for(int64_t N, int64_t K, int32_t kind) {
 }
 
 template <int BN, int KIND>
-nvfp4_status launch_gemm(DeviceState* st, const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& args,
-                         cudaStream_t stream) {
+nvfp4_status launch_gemm(DeviceState* st, const CUtensorMap& ma, const CUtensorMap& mb, const OutMaps& om,
+                         const GemmArgs& args, cudaStream_t stream) {
   using C = GemmCfg<BN>;
   auto kernel = nvfp4_gemm_kernel<BN, KIND>;
   bool& attr = st->smem_attr_set[BN == 256 ? 1 : 0][KIND];
@@ -196,7 +227,7 @@ nvfp4_status launch_gemm(DeviceState* st, const CUtensorMap& ma, const CUtensorM
     attr = true;
   }
   const int grid = args.num_units < st->sm_count ? args.num_units : st->sm_count;
-  kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, args);
+  kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, om, args);
   return launch_status();
 }
 
@@ -345,6 +376,8 @@ nvfp4_status linear_impl(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvf
   CUtensorMap ma, mb;
   if (nvfp4_status e = make_code_map(&ma, a)) return e;
   if (nvfp4_status e = make_code_map(&mb, w)) return e;
+  OutMaps om;
+  if (nvfp4_status e = make_store_maps(&om, out_bf16, ld_out, epi->out_nvfp4 ? out_fp4 : nullptr, M, n_out)) return e;
 
   GemmArgs g{};
   g.M = static_cast<int32_t>(M);
@@ -401,12 +434,12 @@ nvfp4_status linear_impl(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvf
   }
   switch (epi->kind) {
     case NVFP4_EPI_BIAS:
-      return BN == 256 ? launch_gemm<256, kEpiBias>(st, ma, mb, g, s) : launch_gemm<128, kEpiBias>(st, ma, mb, g, s);
+      return BN == 256 ? launch_gemm<256, kEpiBias>(st, ma, mb, om, g, s) : launch_gemm<128, kEpiBias>(st, ma, mb, om, g, s);
     case NVFP4_EPI_RESID_GATE:
-      return BN == 256 ? launch_gemm<256, kEpiResidGate>(st, ma, mb, g, s)
-                       : launch_gemm<128, kEpiResidGate>(st, ma, mb, g, s);
-    case NVFP4_EPI_QKNORM: return launch_gemm<256, kEpiQkNorm>(st, ma, mb, g, s);
-    case NVFP4_EPI_GATED_SILU: return launch_gemm<256, kEpiGatedSilu>(st, ma, mb, g, s);
+      return BN == 256 ? launch_gemm<256, kEpiResidGate>(st, ma, mb, om, g, s)
+                       : launch_gemm<128, kEpiResidGate>(st, ma, mb, om, g, s);
+    case NVFP4_EPI_QKNORM: return launch_gemm<256, kEpiQkNorm>(st, ma, mb, om, g, s);
+    case NVFP4_EPI_GATED_SILU: return launch_gemm<256, kEpiGatedSilu>(st, ma, mb, om, g, s);
   }
   return NVFP4_ERR_INVALID_ARG;
 }
