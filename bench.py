@@ -40,6 +40,40 @@ NOMINAL_FP4_TFLOPS = 9000.0   # NVIDIA's dense FP4 figure for B200
 BF16_TO_FP4 = 4.0             # nominal dense FP4 / dense bf16 tensor-core rate (9 / 2.25)
 
 
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "nvfp4_gemm_up_dram_2048sq.md")
+
+
+def library_sources_sha256():
+    """sha256 over the library's CUDA sources and header (file name, then bytes, in sorted path order)."""
+    import glob
+    import hashlib
+    files = sorted(glob.glob(os.path.join(ROOT, "epilogue_gemm_nvfp4_b200", "csrc", "*.cu*")))
+    files.append(os.path.join(ROOT, "include", "nvfp4.h"))
+    h = hashlib.sha256()
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic():
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, or None when the
+    library's sources have changed since those counters were taken."""
+    try:
+        fields = {}
+        with open(TRAFFIC_PROFILE) as fh:
+            for line in fh:
+                if ":" in line:
+                    k, v = line.split(":", 1)
+                    fields[k.strip()] = v.strip()
+        if fields.get("sources_sha256") != library_sources_sha256():
+            return None
+        return int(fields["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -297,7 +331,9 @@ def run_native(args, ws, rank, local):
                      "frac": round(achieved / peak_fp4, 4),
                      "peak_note": f"{pk['src']} sustained bf16 {pk['bf16_sus']} x {BF16_TO_FP4} (nominal FP4/bf16)",
                      "frac_of_nominal_9pf": round(achieved / NOMINAL_FP4_TFLOPS, 4),
-                     "traffic": None},
+                     "traffic": measured_traffic(),
+                     "traffic_note": "bytes per launch, ncu dram read+write of the full-size launch "
+                                     "(profiles/nvfp4_gemm_up_dram_2048sq.md); null once the kernel sources change"},
         "quantize_roofline": None,
         "e2e": {"value": round(step_flops * ws / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
