@@ -48,6 +48,7 @@ static_assert(kStageKSteps == 2 || kStageKSteps == 4, "stage depth");
 struct GemmArgs {
   int32_t M, N, K;
   int32_t num_m_blocks, num_n_blocks, num_tiles;
+  int32_t num_m_pairs;   // 256-row blocks (CTA-pair kernel)
   int32_t k_steps;      // K / 64
   int32_t k_atoms;      // scale atoms along K (= K / 64)
   const uint8_t* sfa;
@@ -192,11 +193,12 @@ __device__ __forceinline__ void xpose_acquire() {
   __syncwarp();
 }
 
-// Hand the warp's buffer to the TMA engine as the box at (x, y) of `map`.
-__device__ __forceinline__ void xpose_release(const CUtensorMap* map, const uint8_t* xpose, int x, int y) {
+// Hand the warp's buffer to the TMA engine as the box at (x, y) of `map` (nothing to store when the
+// box starts at or past the last row).
+__device__ __forceinline__ void xpose_release(const CUtensorMap* map, const uint8_t* xpose, int x, int y, int rows) {
   fence_proxy_async_smem();  // this thread's shared-memory writes become visible to the TMA engine
   __syncwarp();
-  if ((threadIdx.x & 31) == 0) {
+  if ((threadIdx.x & 31) == 0 && y < rows) {
     tma_store_2d(map, xpose, x, y);
     bulk_commit_group();
   }
@@ -205,7 +207,7 @@ __device__ __forceinline__ void xpose_release(const CUtensorMap* map, const uint
 // Store 16 bf16 values of this lane's row at column col0: lane i writes row i of the 32 x 32-byte box
 // in the 32-byte swizzle (the two 16-byte halves swap every 4 rows, which also keeps the shared-memory
 // writes free of bank conflicts), then the box goes out with one TMA store.
-__device__ __forceinline__ void store_row16_bf16(const OutMaps* om, uint8_t* xpose, int row0, int col0,
+__device__ __forceinline__ void store_row16_bf16(const OutMaps* om, uint8_t* xpose, int row0, int col0, int rows,
                                                  const uint32_t* w) {
   const int lane = threadIdx.x & 31;
   const int sw = (lane >> 2) & 1;
@@ -213,7 +215,7 @@ __device__ __forceinline__ void store_row16_bf16(const OutMaps* om, uint8_t* xpo
   uint4* mine = reinterpret_cast<uint4*>(xpose + lane * 32);
   mine[sw] = make_uint4(w[0], w[1], w[2], w[3]);
   mine[sw ^ 1] = make_uint4(w[4], w[5], w[6], w[7]);
-  xpose_release(&om->out, xpose, col0, row0);
+  xpose_release(&om->out, xpose, col0, row0, rows);
 }
 
 // 32 consecutive output values of one row: bf16 (RNE) output and, when requested, the NVFP4
@@ -224,8 +226,8 @@ __device__ __forceinline__ void emit_row32(const GemmArgs& a, const OutMaps* om,
 #pragma unroll
   for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(o[2 * i], o[2 * i + 1]);
   if (a.out != nullptr) {
-    store_row16_bf16(om, xpose, row0, col0, packed);
-    store_row16_bf16(om, xpose, row0, col0 + 16, packed + 8);
+    store_row16_bf16(om, xpose, row0, col0, a.M, packed);
+    store_row16_bf16(om, xpose, row0, col0 + 16, a.M, packed + 8);
   }
   if (a.q_codes != nullptr) {
     // codes and scales of this row's two 16-blocks; rows at or past M get zero scales (the padding
@@ -258,9 +260,10 @@ __device__ __forceinline__ void emit_row32(const GemmArgs& a, const OutMaps* om,
     const int lane = threadIdx.x & 31;
     xpose_acquire();
     *reinterpret_cast<uint4*>(xpose + lane * 16) = make_uint4(words[0], words[1], words[2], words[3]);
-    xpose_release(&om->q_codes, xpose, col0 / 2, row0);
-    *reinterpret_cast<uint16_t*>(a.q_scales + scale_offset(row, col0 / 16, a.q_k_atoms)) =
-        static_cast<uint16_t>(sc[0] | (sc[1] << 8));
+    xpose_release(&om->q_codes, xpose, col0 / 2, row0, a.M);
+    if (row < a.num_m_blocks * 128)  // the scale layout's rows end at the 128-row padding
+      *reinterpret_cast<uint16_t*>(a.q_scales + scale_offset(row, col0 / 16, a.q_k_atoms)) =
+          static_cast<uint16_t>(sc[0] | (sc[1] << 8));
   }
 }
 

@@ -11,6 +11,7 @@
 
 #include "nvfp4.h"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "ptx.cuh"
 #include "quantize.cuh"
 
@@ -27,6 +28,7 @@ struct DeviceState {
   int sm_count = 0;
   unsigned int* error_word = nullptr;
   bool smem_attr_set[2][4] = {};
+  int pair_clusters[4] = {};  // resident CTA pairs per epilogue kind (0 until first use)
 };
 
 std::mutex g_mutex;
@@ -215,6 +217,38 @@ int tile_n_for(int64_t N, int64_t K, int32_t kind) {
   return 0;
 }
 
+// 256-wide tiles without split-K run on CTA pairs unless NVFP4_GEMM_PAIR=0.
+bool pair_kernel_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("NVFP4_GEMM_PAIR");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
+
+template <int KIND>
+nvfp4_status launch_gemm_pair(DeviceState* st, const CUtensorMap& ma, const CUtensorMap& mb, const OutMaps& om,
+                              const GemmArgs& args, cudaStream_t stream) {
+  using C = GemmPairCfg;
+  auto kernel = nvfp4_gemm_pair_kernel<KIND>;
+  int& clusters = st->pair_clusters[KIND];
+  if (clusters == 0) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    // clusters that can be resident at once: the persistent grid must not exceed one wave
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (st->sm_count / 2));
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n < 1) return NVFP4_ERR_CUDA;
+    clusters = n;
+  }
+  const int grid_clusters = args.num_units < clusters ? args.num_units : clusters;
+  kernel<<<2 * grid_clusters, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, om, args);
+  return launch_status();
+}
+
 template <int BN, int KIND>
 nvfp4_status launch_gemm(DeviceState* st, const CUtensorMap& ma, const CUtensorMap& mb, const OutMaps& om,
                          const GemmArgs& args, cudaStream_t stream) {
@@ -386,6 +420,7 @@ nvfp4_status linear_impl(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvf
   g.num_m_blocks = static_cast<int32_t>((M + 127) / 128);
   g.num_n_blocks = static_cast<int32_t>(epi->kind == NVFP4_EPI_GATED_SILU ? (N / 2) / 128 : N / BN);
   g.num_tiles = g.num_m_blocks * g.num_n_blocks;
+  g.num_m_pairs = static_cast<int32_t>((M + 255) / 256);
   g.k_steps = static_cast<int32_t>(K / 64);
   g.k_atoms = static_cast<int32_t>(k_atoms_of(K));
   g.sfa = static_cast<const uint8_t*>(a->scales);
@@ -431,6 +466,17 @@ nvfp4_status linear_impl(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvf
     g.split_flags = static_cast<unsigned int*>(ws);
     g.split_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + flag_bytes);
     if (cudaMemsetAsync(ws, 0, static_cast<size_t>(g.num_tiles) * 4, s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  }
+  if (BN == 256 && g.splits == 1 && pair_kernel_enabled()) {
+    g.num_tiles = g.num_m_pairs * g.num_n_blocks;
+    g.num_units = g.num_tiles;
+    switch (epi->kind) {
+      case NVFP4_EPI_BIAS: return launch_gemm_pair<kEpiBias>(st, ma, mb, om, g, s);
+      case NVFP4_EPI_RESID_GATE: return launch_gemm_pair<kEpiResidGate>(st, ma, mb, om, g, s);
+      case NVFP4_EPI_QKNORM: return launch_gemm_pair<kEpiQkNorm>(st, ma, mb, om, g, s);
+      case NVFP4_EPI_GATED_SILU: return launch_gemm_pair<kEpiGatedSilu>(st, ma, mb, om, g, s);
+    }
+    return NVFP4_ERR_INVALID_ARG;
   }
   switch (epi->kind) {
     case NVFP4_EPI_BIAS:
