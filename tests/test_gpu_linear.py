@@ -5,6 +5,8 @@ bit-exact against that quantisation first, so both sides multiply the same NVFP4
 for GEMM + epilogue outputs is a normwise max relative error of 2e-2 (bf16 output).  Row independence
 is checked bitwise on the GPU.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -113,8 +115,11 @@ def test_resid_gate_small(lib):
     check(f32(out), ref["y"], "resid_gate")
 
 
-def test_gated_silu_with_requant_small(lib):
-    case = W.case_ffn_up(130, K=512, F=256, seed=7)
+@pytest.mark.parametrize("M", [130, 100])
+def test_gated_silu_with_requant_small(lib, M):
+    # M = 100: on CTA pairs the second CTA's 128-row block lies wholly past M and past the scale
+    # layout's padded rows, so it must write nothing
+    case = W.case_ffn_up(M, K=512, F=256, seed=7)
     case.bias = W.to_bf16(np.random.default_rng(70).standard_normal(512).astype(np.float32) * 0.01)
     a_ref, w_ref, ref = run_oracle(case)
     g_out = np.float32(np.max(np.abs(ref["bf16"])) / np.float32(2688.0))
@@ -243,3 +248,30 @@ def test_text_projection_sampled(lib, T):
     rows = np.arange(T) if T == 512 else sample_rows(T, n=40, seed=2)
     _, _, ref = run_oracle(case, rows=rows)
     check(f32(out)[rows], ref["y"], f"text T={T}")
+
+
+def test_one_cta_and_pair_kernels_agree(lib, tmp_path):
+    """256-wide tiles run on CTA pairs by default; NVFP4_GEMM_PAIR=0 selects the one-CTA kernel.
+    Both follow the oracle, and they give the same bits: the K order of every output is the same."""
+    import subprocess
+    import sys
+    script = tmp_path / "one_cta.py"
+    out_path = tmp_path / "one_cta.npy"
+    script.write_text(
+        "import sys, numpy as np, torch\n"
+        f"sys.path.insert(0, {repr(os.path.dirname(os.path.dirname(os.path.abspath(__file__))))})\n"
+        "from tests.test_gpu_linear import run_gpu, f32\n"
+        "from epilogue_gemm_nvfp4_b200 import workloads as W\n"
+        "case = W.case_qkv(300, n_heads=2, K=768, seed=11)\n"
+        "_, _, out = run_gpu(case)\n"
+        f"np.save({repr(str(out_path))}, f32(out))\n")
+    env = dict(os.environ, NVFP4_GEMM_PAIR="0")
+    subprocess.run([sys.executable, str(script)], check=True, env=env, timeout=300)
+    one = np.load(out_path)
+    case = W.case_qkv(300, n_heads=2, K=768, seed=11)
+    _, _, out = run_gpu(case)
+    pair = f32(out)
+    _, _, ref = run_oracle(case)
+    check(one, ref["y"], "one-CTA kernel")
+    check(pair, ref["y"], "pair kernel")
+    assert np.array_equal(one, pair)
