@@ -244,7 +244,7 @@ class BlockSet:
         B.linear(self.up_q, self.wq["down"], "resid_gate", residual=self.res, gate=self.gate, out=self.out["down"])
         mark("down", 1)
 
-    LAUNCHES_PER_STEP = 3 * 3 + 4   # per activation: amax, quantise, finalise; four GEMMs
+    LAUNCHES_PER_STEP = 3 * 2 + 4   # per activation: amax (which also writes g), quantise; four GEMMs
 
 
 OPS = ("quant_qkv", "qkv", "quant_out", "out", "quant_up", "up", "down")

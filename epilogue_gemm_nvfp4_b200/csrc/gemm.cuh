@@ -218,16 +218,35 @@ __device__ __forceinline__ void store_row16_bf16(const OutMaps* om, uint8_t* xpo
   xpose_release(&om->out, xpose, col0, row0, rows);
 }
 
+// Store 32 bf16 values of this lane's row at column col0 as one 32-row x 64-byte box in the 64-byte
+// swizzle (16-byte chunk j of row r sits at chunk j ^ ((r >> 1) & 3), which keeps the shared-memory
+// writes at four wavefronts): half the TMA store operations of two 16-column boxes.  Needs a 2 KB box.
+__device__ __forceinline__ void store_row32_bf16(const OutMaps* om, uint8_t* xpose, int row0, int col0, int rows,
+                                                 const uint32_t* w) {
+  const int lane = threadIdx.x & 31;
+  const int sw = (lane >> 1) & 3;
+  xpose_acquire();
+  uint4* mine = reinterpret_cast<uint4*>(xpose + lane * 64);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) mine[j ^ sw] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  xpose_release(&om->out, xpose, col0, row0, rows);
+}
+
 // 32 consecutive output values of one row: bf16 (RNE) output and, when requested, the NVFP4
 // re-quantisation of those bf16 values with the caller's tensor scale (the quantiser's block rule).
+template <int kBoxBytes>
 __device__ __forceinline__ void emit_row32(const GemmArgs& a, const OutMaps* om, uint8_t* xpose, int row0, int row,
                                            int col0, const float* o, float qg) {
   uint32_t packed[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(o[2 * i], o[2 * i + 1]);
   if (a.out != nullptr) {
-    store_row16_bf16(om, xpose, row0, col0, a.M, packed);
-    store_row16_bf16(om, xpose, row0, col0 + 16, a.M, packed + 8);
+    if constexpr (kBoxBytes >= 2048) {
+      store_row32_bf16(om, xpose, row0, col0, a.M, packed);
+    } else {
+      store_row16_bf16(om, xpose, row0, col0, a.M, packed);
+      store_row16_bf16(om, xpose, row0, col0 + 16, a.M, packed + 8);
+    }
   }
   if (a.q_codes != nullptr) {
     // codes and scales of this row's two 16-blocks; rows at or past M get zero scales (the padding
@@ -271,7 +290,8 @@ __device__ __forceinline__ void emit_row32(const GemmArgs& a, const OutMaps* om,
 // epilogue: registers <- TMEM, release, then math and stores
 // ------------------------------------------------------------------------------------------
 
-template <int BN, int KIND>
+// kBoxBytes: the per-warp shared-memory store box, 1 KB (32 x 16 bf16) or 2 KB (32 x 32 bf16).
+template <int BN, int KIND, int kBoxBytes = 1024>
 struct Epilogue {
   static constexpr int COLS = (KIND == kEpiGatedSilu) ? 128 : BN / 2;  // accumulator columns per thread
 
@@ -339,7 +359,7 @@ struct Epilogue {
             o[16 * g + i] = __fdividef(ya, 1.0f + __expf(-ya)) * yb;  // silu(a) * b
           }
         }
-        emit_row32(a, om, xpose, row0, row, ocol, o, qg);
+        emit_row32<kBoxBytes>(a, om, xpose, row0, row, ocol, o, qg);
       }
     } else {
       const int col_e = nb * BN + COLS * e;
@@ -380,7 +400,7 @@ struct Epilogue {
             }
           }
         }
-        emit_row32(a, om, xpose, row0, row, col0, y, qg);
+        emit_row32<kBoxBytes>(a, om, xpose, row0, row, col0, y, qg);
       }
     }
   }

@@ -42,7 +42,7 @@ struct GemmPairCfg {
   static constexpr int SF_COLS = SFA_COLS + SFB_COLS;
   static constexpr int TMEM_COLS = 512;
   static constexpr int EPI_WARPS = 8;
-  static constexpr int XPOSE_BYTES = 1024;
+  static constexpr int XPOSE_BYTES = 2048;             // per epilogue warp: 32 rows x 64 bytes
   static constexpr int AUX_BYTES = 1536;
   static constexpr int SS_OFFSET = 512;
   static constexpr int SMEM_LIMIT = 232448;
@@ -58,7 +58,7 @@ struct GemmPairCfg {
   static_assert((3 * STAGES + 5) * 8 + 16 <= SS_OFFSET, "barrier area");
   static_assert((SMEM_LIMIT >> 4) < (1 << 14), "operand descriptors advance by adds inside the 14-bit address field");
   // the epilogue and its column split are those of the one-CTA 256-wide tile
-  static_assert(GemmCfg<256>::EPI_WARPS == EPI_WARPS && GemmCfg<256>::XPOSE_BYTES == XPOSE_BYTES, "epilogue");
+  static_assert(GemmCfg<256>::EPI_WARPS == EPI_WARPS, "epilogue");
 };
 
 struct PairUnit {
@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(512, 1) __cluster_dims__(2, 1, 1)
     nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                            const __grid_constant__ OutMaps out_maps, const __grid_constant__ GemmArgs args) {
   using C = GemmPairCfg;
-  using E = Epilogue<256, KIND>;
+  using E = Epilogue<256, KIND, C::XPOSE_BYTES>;
   extern __shared__ uint8_t smem_raw[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw);
   uint64_t* empty = full + C::STAGES;

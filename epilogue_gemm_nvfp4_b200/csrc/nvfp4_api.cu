@@ -80,6 +80,29 @@ nvfp4_status scratch_for(cudaStream_t s, size_t need, void** out) {
   return NVFP4_OK;
 }
 
+// Per-(device, stream) state of the dynamic-scale quantiser's amax reduction: {amax bits, CTAs done},
+// zero between calls (each call's last CTA clears it).  Allocated and cleared on the stream's first
+// dynamic-scale call, which therefore must not run under graph capture.
+std::map<std::pair<int, uintptr_t>, unsigned int*> g_amax_state;
+
+nvfp4_status amax_state_for(cudaStream_t s, unsigned int** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  unsigned int*& p = g_amax_state[{dev, reinterpret_cast<uintptr_t>(s)}];
+  if (p == nullptr) {
+    void* q = nullptr;
+    if (cudaMalloc(&q, 256) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (cudaMemsetAsync(q, 0, 256, s) != cudaSuccess) {
+      cudaFree(q);
+      return NVFP4_ERR_CUDA;
+    }
+    p = static_cast<unsigned int*>(q);
+  }
+  *out = p;
+  return NVFP4_OK;
+}
+
 // Per-device set-up, done once with that device current: SM count and the address of the error word.
 nvfp4_status device_state(DeviceState** out) {
   int dev = 0;
@@ -173,10 +196,11 @@ nvfp4_status make_code_map(CUtensorMap* map, const nvfp4_tensor* t) {
 }
 
 // TMA store maps of the fused linear's outputs, in the boxes the epilogue writes (32 rows of one warp):
-// bf16 output 16 columns wide with the 32-byte swizzle of its shared-memory buffer, E2M1 codes 16
-// bytes wide unswizzled.  A map stays zeroed when its output is not requested (the kernel never uses it).
+// bf16 output `box_cols` (16 or 32) columns wide with the 32- or 64-byte swizzle of its shared-memory
+// box, E2M1 codes 16 bytes wide unswizzled.  A map stays zeroed when its output is not requested (the
+// kernel never uses it).
 nvfp4_status make_store_maps(OutMaps* om, void* out_bf16, int64_t ld_out, const nvfp4_tensor* out_fp4, int64_t M,
-                             int64_t n_out) {
+                             int64_t n_out, int box_cols) {
   std::memset(om, 0, sizeof(*om));
   auto encode = tensor_map_encoder();
   if (!encode) return NVFP4_ERR_CUDA;
@@ -184,9 +208,10 @@ nvfp4_status make_store_maps(OutMaps* om, void* out_bf16, int64_t ld_out, const 
   if (out_bf16) {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(n_out), static_cast<cuuint64_t>(M)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_out * 2)};
-    cuuint32_t box[2] = {16, 32};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), 32};
     if (encode(&om->out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out_bf16, dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return NVFP4_ERR_CUDA;
   }
@@ -330,20 +355,18 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
   const int64_t tasks = rows * ((steps + kQuantStepsPerTask - 1) / kQuantStepsPerTask) + 1;
   // one 256-bit load per block when every block starts on a 32-byte boundary
   const bool vec32 = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx * 2) % 32 == 0;
-  auto qk = compute_scale ? (vec32 ? quantize_kernel<true, true, true> : quantize_kernel<true, true, false>)
-                          : (vec32 ? quantize_kernel<false, false, true> : quantize_kernel<false, false, false>);
+  // dynamic scale: the amax pass (which also writes g) streams the tensor front to back, then the
+  // quantiser walks it back to front so that its first tasks re-read from L2 what that pass left there
+  auto qk = compute_scale ? (vec32 ? quantize_kernel<true, true> : quantize_kernel<true, false>)
+                          : (vec32 ? quantize_kernel<false, true> : quantize_kernel<false, false>);
   const int qgrid = resident_grid(qk, 256, tasks, 8, st->sm_count);
   if (compute_scale) {
-    if (cudaMemsetAsync(out->tensor_scale, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
-    if (rows > 0) {
-      const int agrid = resident_grid(amax_kernel, 256, rows * cols / 8, 256 * 4, st->sm_count);
-      amax_kernel<<<agrid, 256, 0, s>>>(xb, rows, cols, ldx, reinterpret_cast<unsigned int*>(out->tensor_scale));
-    }
-    qk<<<qgrid, 256, 0, s>>>(xb, rows, cols, ldx, out->tensor_scale, codes, ld, scales, ka);
-    finalize_scale_kernel<<<1, 1, 0, s>>>(out->tensor_scale);
-  } else {
-    qk<<<qgrid, 256, 0, s>>>(xb, rows, cols, ldx, out->tensor_scale, codes, ld, scales, ka);
+    unsigned int* state = nullptr;
+    if (nvfp4_status e = amax_state_for(s, &state)) return e;
+    const int agrid = resident_grid(amax_scale_kernel, 256, rows * cols / 8, 256 * 4, st->sm_count);
+    amax_scale_kernel<<<agrid, 256, 0, s>>>(xb, rows, cols, ldx, state, out->tensor_scale);
   }
+  qk<<<qgrid, 256, 0, s>>>(xb, rows, cols, ldx, out->tensor_scale, codes, ld, scales, ka);
   return launch_status();
 }
 
@@ -410,8 +433,11 @@ nvfp4_status linear_impl(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvf
   CUtensorMap ma, mb;
   if (nvfp4_status e = make_code_map(&ma, a)) return e;
   if (nvfp4_status e = make_code_map(&mb, w)) return e;
+  const bool pair = BN == 256 && split_k_for(K, epi->kind) == 1 && pair_kernel_enabled();
   OutMaps om;
-  if (nvfp4_status e = make_store_maps(&om, out_bf16, ld_out, epi->out_nvfp4 ? out_fp4 : nullptr, M, n_out)) return e;
+  if (nvfp4_status e = make_store_maps(&om, out_bf16, ld_out, epi->out_nvfp4 ? out_fp4 : nullptr, M, n_out,
+                                       pair ? GemmPairCfg::XPOSE_BYTES / 64 : 16))
+    return e;
 
   GemmArgs g{};
   g.M = static_cast<int32_t>(M);
@@ -467,7 +493,7 @@ nvfp4_status linear_impl(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvf
     g.split_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + flag_bytes);
     if (cudaMemsetAsync(ws, 0, static_cast<size_t>(g.num_tiles) * 4, s) != cudaSuccess) return NVFP4_ERR_CUDA;
   }
-  if (BN == 256 && g.splits == 1 && pair_kernel_enabled()) {
+  if (pair) {
     g.num_tiles = g.num_m_pairs * g.num_n_blocks;
     g.num_units = g.num_tiles;
     switch (epi->kind) {

@@ -32,8 +32,9 @@ __device__ __forceinline__ uint32_t bf16x2_absmax_bits(uint32_t w) {
 // so the reduction runs on integers and one atomicMax per CTA publishes the fp32 bit pattern.
 // ------------------------------------------------------------------------------------------
 
-__global__ void __launch_bounds__(256) amax_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
-                                                   int64_t cols, int64_t ldx, unsigned int* __restrict__ out_bits) {
+// max over this CTA's share of the matrix of the bf16 magnitude bits (valid in thread 0)
+__device__ __forceinline__ uint32_t block_absmax_bits(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols,
+                                                      int64_t ldx) {
   uint32_t m = 0;
   const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -71,22 +72,37 @@ __global__ void __launch_bounds__(256) amax_kernel(const __nv_bfloat16* __restri
   __shared__ uint32_t red[8];
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0)
     for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) m = max(m, red[w]);
-    if (m) atomicMax(out_bits, m << 16);  // bf16 magnitude -> fp32 bit pattern
+  return m;
+}
+
+__global__ void __launch_bounds__(256) amax_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
+                                                   int64_t cols, int64_t ldx, unsigned int* __restrict__ out_bits) {
+  const uint32_t m = block_absmax_bits(x, rows, cols, ldx);
+  if (threadIdx.x == 0 && m) atomicMax(out_bits, m << 16);  // bf16 magnitude -> fp32 bit pattern
+}
+
+// The same reduction, finished in place: the last CTA to finish writes the tensor decode scale
+// g = amax / 2688 (1 for an all-zero tensor).  `state` is the caller's per-stream pair {amax bits,
+// CTAs done}, zero on entry; the last CTA puts it back to zero for the next call on the stream.  Each
+// CTA publishes its max before it takes its ticket (atomicMax, fence, atomicAdd), so the CTA that draws
+// the last ticket sees every CTA's max.
+__global__ void __launch_bounds__(256) amax_scale_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
+                                                         int64_t cols, int64_t ldx, unsigned int* __restrict__ state,
+                                                         float* __restrict__ tensor_scale) {
+  const uint32_t m = block_absmax_bits(x, rows, cols, ldx);
+  if (threadIdx.x == 0) {
+    if (m) atomicMax(&state[0], m << 16);
+    __threadfence();
+    if (atomicAdd(&state[1], 1u) == gridDim.x - 1) {
+      __threadfence();
+      const float amax = __uint_as_float(atomicOr(&state[0], 0u));
+      *tensor_scale = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, kTensorScaleDivisor);
+      state[0] = 0u;
+      state[1] = 0u;
+    }
   }
-}
-
-// g = amax / 2688 (or 1 for an all-zero tensor), in place: the slot held amax bits.
-__global__ void finalize_scale_kernel(float* __restrict__ slot) {
-  const float amax = *slot;
-  *slot = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, kTensorScaleDivisor);
-}
-
-__device__ __forceinline__ float tensor_scale_from(const float* src, bool from_amax) {
-  const float v = *src;
-  if (!from_amax) return v;
-  return (v == 0.0f) ? 1.0f : __fdiv_rn(v, kTensorScaleDivisor);
 }
 
 // The block rule for one 16-element block, given its amax and the tensor decode scale g:
@@ -124,12 +140,12 @@ __device__ __forceinline__ void ld_block32(const __nv_bfloat16* p, bool vec32, u
   }
 }
 
-template <bool kFromAmax, bool kReverse, bool kVec32>
+template <bool kReverse, bool kVec32>
 __global__ void __launch_bounds__(256, 6) quantize_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
                                                        int64_t cols, int64_t ldx, const float* __restrict__ scale_src,
                                                        uint8_t* __restrict__ codes, int64_t ld_codes,
                                                        uint8_t* __restrict__ scales, int64_t k_atoms) {
-  const float g = tensor_scale_from(scale_src, kFromAmax);
+  const float g = *scale_src;
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   const int64_t gwarp = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);

@@ -122,11 +122,14 @@ typedef struct {
 /*
  * Quantise a bf16 matrix x [rows, cols] (row stride ldx elements) to NVFP4 into `out`
  * (out->rows == rows, out->cols == cols).
- *   compute_scale = 1: compute g = amax(|x|) / 2688 on the device and store it in *out->tensor_scale
- *                      (an amax pass, the quantise pass and a one-thread finalise, stream-ordered).
+ *   compute_scale = 1: compute g = amax(|x|) / 2688 (1 when x is all zeros or empty) on the device and
+ *                      store it in *out->tensor_scale: two stream-ordered kernels, an amax pass whose
+ *                      last CTA writes g, then the quantise pass.  The first such call on a stream
+ *                      allocates 256 bytes of per-stream reduction state, so it must not be the first
+ *                      call made under CUDA graph capture.
  *   compute_scale = 0: use the g already stored in *out->tensor_scale (a calibrated static scale).
  * Rules: cols % 16 == 0; x, ldx*2, codes and scales 16-byte aligned; ld_codes a multiple of 8.
- * rows == 0 is a no-op.
+ * rows == 0 writes no codes.
  */
 NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int32_t compute_scale,
                             const nvfp4_tensor* out, nvfp4_stream_t stream);

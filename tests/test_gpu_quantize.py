@@ -89,3 +89,21 @@ def test_quantize_bitexact_workload_tensors(lib, name):
     for t in tensors:
         q = B.quantize(t.cuda())
         assert_quant_bitexact(q, oracle_quantize(t), *t.shape)
+
+
+def test_dynamic_scale_state_is_per_call_and_per_stream(lib):
+    """The dynamic scale's amax reduction keeps {amax, CTAs done} per stream and clears it in the last
+    CTA: a large tensor followed by a 100x smaller one on the same stream, and a call on a second
+    stream, each get their own g."""
+    rng = np.random.default_rng(41)
+    big = W.to_bf16(rng.standard_normal((300, 512)).astype(np.float32) * 50.0)
+    small = W.to_bf16(rng.standard_normal((300, 512)).astype(np.float32) * 0.5)
+    ref = {id(big): oracle_quantize(big), id(small): oracle_quantize(small)}
+    for x in (big, small, big, small):
+        assert_quant_bitexact(B.quantize(x.cuda()), ref[id(x)], 300, 512)
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        q = B.quantize(small.cuda())
+    side.synchronize()
+    assert_quant_bitexact(q, ref[id(small)], 300, 512)
+    assert_quant_bitexact(B.quantize(big.cuda()), ref[id(big)], 300, 512)
