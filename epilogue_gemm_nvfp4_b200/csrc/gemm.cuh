@@ -166,6 +166,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&p);
 }
 
+// silu(a) = a * sigmoid(a) = h + h * tanh(h) with h = a / 2: one hardware tanh (tanh.approx.f32,
+// relative error about 2^-11, far below the bf16 output's 2^-8) instead of an exponential and a
+// reciprocal.
+__device__ __forceinline__ float silu(float a) {
+  const float h = 0.5f * a;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+  return fmaf(h, t, h);
+}
+
 __device__ __forceinline__ void tmem_load32(uint32_t taddr, float* v) {
   uint32_t r[32];
   tmem_ld_32x32b_x32(taddr, r);
@@ -356,7 +366,7 @@ struct Epilogue {
               ya += ba[i];
               yb += bb[i];
             }
-            o[16 * g + i] = __fdividef(ya, 1.0f + __expf(-ya)) * yb;  // silu(a) * b
+            o[16 * g + i] = silu(ya) * yb;
           }
         }
         emit_row32<kBoxBytes>(a, om, xpose, row0, row, ocol, o, qg);
