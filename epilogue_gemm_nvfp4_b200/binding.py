@@ -36,7 +36,7 @@ class CEpilogue(ctypes.Structure):
                 ("gamma_k", ctypes.c_void_p), ("eps", ctypes.c_float), ("head_dim", ctypes.c_int32),
                 ("q_col0", ctypes.c_int64), ("k_col0", ctypes.c_int64), ("qk_cols", ctypes.c_int64),
                 ("residual", ctypes.c_void_p), ("ld_residual", ctypes.c_int64), ("gate", ctypes.c_void_p),
-                ("out_nvfp4", ctypes.c_int32)]
+                ("out_nvfp4", ctypes.c_int32), ("out_amax", ctypes.c_void_p)]
 
 
 class NvFp4Error(RuntimeError):
@@ -173,10 +173,13 @@ def amax(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch
 
 
 def make_epilogue(kind: str = "bias", bias=None, gamma_q=None, gamma_k=None, eps=1e-6, q_col0=0, k_col0=0,
-                  qk_cols=0, head_dim=256, residual=None, gate=None, out_nvfp4=False) -> CEpilogue:
+                  qk_cols=0, head_dim=256, residual=None, gate=None, out_nvfp4=False, out_amax=None) -> CEpilogue:
+    """``out_amax``: fp32 device tensor of one element (zeroed by the caller) that the kernel raises to
+    max |bf16 output|."""
     return CEpilogue(EPI_KINDS[kind], _ptr(bias), _ptr(gamma_q), _ptr(gamma_k), float(eps), int(head_dim),
                      int(q_col0), int(k_col0), int(qk_cols), _ptr(residual),
-                     residual.stride(0) if residual is not None else 0, _ptr(gate), int(bool(out_nvfp4)))
+                     residual.stride(0) if residual is not None else 0, _ptr(gate), int(bool(out_nvfp4)),
+                     _ptr(out_amax))
 
 
 def linear(a: QTensor, w: QTensor, kind: str = "bias", bias=None, out: torch.Tensor | None = None,

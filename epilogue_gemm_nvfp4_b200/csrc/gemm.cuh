@@ -70,6 +70,7 @@ struct GemmArgs {
   uint8_t* q_scales;
   const float* q_g;
   int32_t q_k_atoms;
+  unsigned int* out_amax_bits;  // raised to max |bf16 output| (fp32 bit pattern), or nullptr
   unsigned int* error_word;
   uint64_t timeout_ns;
   // split-K: `splits` consecutive work units share one output tile, each summing a contiguous range
@@ -246,10 +247,16 @@ __device__ __forceinline__ void store_row32_bf16(const OutMaps* om, uint8_t* xpo
 // re-quantisation of those bf16 values with the caller's tensor scale (the quantiser's block rule).
 template <int kBoxBytes>
 __device__ __forceinline__ void emit_row32(const GemmArgs& a, const OutMaps* om, uint8_t* xpose, int row0, int row,
-                                           int col0, const float* o, float qg) {
+                                           int col0, const float* o, float qg, uint32_t& amax_bits) {
   uint32_t packed[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(o[2 * i], o[2 * i + 1]);
+  if (a.out_amax_bits != nullptr && row < a.M) {
+    uint32_t m = amax_bits;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = max(m, bf16x2_absmax_bits(packed[i]));
+    amax_bits = m;
+  }
   if (a.out != nullptr) {
     if constexpr (kBoxBytes >= 2048) {
       store_row32_bf16(om, xpose, row0, col0, a.M, packed);
@@ -294,6 +301,14 @@ __device__ __forceinline__ void emit_row32(const GemmArgs& a, const OutMaps* om,
       *reinterpret_cast<uint16_t*>(a.q_scales + scale_offset(row, col0 / 16, a.q_k_atoms)) =
           static_cast<uint16_t>(sc[0] | (sc[1] << 8));
   }
+}
+
+// Publish a warp's largest output magnitude (bf16 magnitude bits) with one atomic max on the fp32
+// bit pattern; every lane of the warp calls this.
+__device__ __forceinline__ void publish_amax(unsigned int* out_bits, uint32_t m) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0 && out_bits != nullptr && m != 0) atomicMax(out_bits, m << 16);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -346,7 +361,7 @@ struct Epilogue {
   static __device__ __forceinline__ void finish(const GemmArgs& a, const OutMaps* om, uint8_t* xpose, int row0, int row,
                                                 int e, int nb,
                                                 float alpha, float qg, const __nv_bfloat16* gamma, float ss,
-                                                float* acc) {
+                                                float* acc, uint32_t& amax_bits) {
     if constexpr (KIND == kEpiGatedSilu) {
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -369,7 +384,7 @@ struct Epilogue {
             o[16 * g + i] = silu(ya) * yb;
           }
         }
-        emit_row32<kBoxBytes>(a, om, xpose, row0, row, ocol, o, qg);
+        emit_row32<kBoxBytes>(a, om, xpose, row0, row, ocol, o, qg, amax_bits);
       }
     } else {
       const int col_e = nb * BN + COLS * e;
@@ -410,7 +425,7 @@ struct Epilogue {
             }
           }
         }
-        emit_row32<kBoxBytes>(a, om, xpose, row0, row, col0, y, qg);
+        emit_row32<kBoxBytes>(a, om, xpose, row0, row, col0, y, qg, amax_bits);
       }
     }
   }
@@ -724,6 +739,7 @@ __global__ void __launch_bounds__(512, 1)
     const float qg = args.q_codes != nullptr ? *args.q_g : 1.0f;
     int abuf = 0;
     uint32_t aphase = 0;
+    uint32_t amax_bits = 0;
     for (int u = blockIdx.x; u < args.num_units; u += gridDim.x) {
       const WorkUnit wu = work_unit(args, u, num_kb);
       const int mb = wu.mb, nb = wu.nb;
@@ -756,8 +772,9 @@ __global__ void __launch_bounds__(512, 1)
         continue;
       float ss = 0.0f;
       if (KIND == kEpiQkNorm && gamma != nullptr) ss = E::head_sumsq(args, e, nb, q * 32 + lane, alpha, acc, ss_x);
-      E::finish(args, &out_maps, xpose, row0, row0 + lane, e, nb, alpha, qg, gamma, ss, acc);
+      E::finish(args, &out_maps, xpose, row0, row0 + lane, e, nb, alpha, qg, gamma, ss, acc, amax_bits);
     }
+    publish_amax(args.out_amax_bits, amax_bits);
     // the TMA stores read this warp's buffer and write the outputs asynchronously: both must be done
     // before the CTA's shared memory is released
     if (lane == 0) bulk_wait_group_all();

@@ -317,6 +317,7 @@ __global__ void __launch_bounds__(512, 1) __cluster_dims__(2, 1, 1)
     const float qg = args.q_codes != nullptr ? *args.q_g : 1.0f;
     const uint32_t leader_acc_empty = cluster_addr(&acc_empty[0], 0);
     uint32_t aphase = 0;
+    uint32_t amax_bits = 0;
     for (int u = cluster; u < args.num_units; u += num_clusters) {
       const PairUnit pu = pair_unit(args, u);
       const int mb = 2 * pu.mp + static_cast<int>(rank);
@@ -343,8 +344,9 @@ __global__ void __launch_bounds__(512, 1) __cluster_dims__(2, 1, 1)
       aphase ^= 1u;
       float ss = 0.0f;
       if (KIND == kEpiQkNorm && gamma != nullptr) ss = E::head_sumsq(args, e, nb, q * 32 + lane, alpha, acc, ss_x);
-      E::finish(args, &out_maps, xpose, row0, row0 + lane, e, nb, alpha, qg, gamma, ss, acc);
+      E::finish(args, &out_maps, xpose, row0, row0 + lane, e, nb, alpha, qg, gamma, ss, acc, amax_bits);
     }
+    publish_amax(args.out_amax_bits, amax_bits);
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
   }

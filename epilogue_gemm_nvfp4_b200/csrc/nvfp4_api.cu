@@ -416,6 +416,7 @@ nvfp4_status linear_impl(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvf
     if (!epi->residual || !epi->gate || epi->ld_residual < n_out) return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(epi->residual) || (epi->ld_residual * 2) % 16 || !aligned16(epi->gate)) return NVFP4_ERR_MISALIGNED;
   }
+  if (epi->out_amax && !aligned4(epi->out_amax)) return NVFP4_ERR_MISALIGNED;
   if (epi->out_nvfp4) {
     if (nvfp4_status e = check_tensor(out_fp4, true, 16)) return e;
     if (out_fp4->rows != M || out_fp4->cols != n_out) return NVFP4_ERR_INVALID_ARG;
@@ -472,6 +473,7 @@ nvfp4_status linear_impl(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvf
     g.q_g = out_fp4->tensor_scale;
     g.q_k_atoms = static_cast<int32_t>(k_atoms_of(n_out));
   }
+  g.out_amax_bits = reinterpret_cast<unsigned int*>(epi->out_amax);
   g.error_word = st->error_word;
   g.timeout_ns = wait_timeout_ns();
   g.splits = split_k_for(K, epi->kind);

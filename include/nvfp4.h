@@ -102,6 +102,12 @@ typedef enum {
  *   out_nvfp4:     1 = also re-quantise the bf16-rounded output to NVFP4 into `out_fp4` with the
  *                  caller's static decode scale already stored in out_fp4->tensor_scale (the rule of
  *                  nvfp4_quantize, so the codes equal nvfp4_quantize of the bf16 output bit for bit).
+ *   out_amax:      device fp32, or NULL.  When given, the kernel raises *out_amax to the largest |y| of
+ *                  the bf16-rounded output (the values out_nvfp4 quantises; rows < M only), as an
+ *                  atomic max on the bit pattern, so *out_amax must hold a non-negative float (0 to
+ *                  start, or a running max over calls).  amax / 2688 is then the decode scale that
+ *                  nvfp4_quantize would compute for this output: a delayed scale for the next call's
+ *                  out_fp4, available without a separate pass over the output.
  */
 typedef struct {
   int32_t kind;
@@ -117,6 +123,7 @@ typedef struct {
   int64_t ld_residual;
   const float* gate;
   int32_t out_nvfp4;
+  float* out_amax;
 } nvfp4_epilogue_desc;
 
 /*

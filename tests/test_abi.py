@@ -96,3 +96,30 @@ def test_valid_call_without_a_device_reports_cuda_error(lib):
     desc = B.CEpilogue()
     assert lib.nvfp4_linear(ctypes.byref(a), ctypes.byref(w), ctypes.byref(desc), 0x10000, 512, None, None) \
         == B.ERR_CUDA
+
+
+def test_ctypes_structs_match_the_header(tmp_path):
+    """The binding's ctypes structs have the C header's field offsets and sizes (compiled with gcc)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    structs = {"nvfp4_tensor": B.CTensor, "nvfp4_epilogue_desc": B.CEpilogue}
+    lines = ['#include <stdio.h>', '#include "nvfp4.h"', "int main(void) {"]
+    for cname, py in structs.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for field, _ in py._fields_:
+            lines.append(f'  printf("{cname} {field} %zu\\n", offsetof({cname}, {field}));')
+    lines.append("  return 0;\n}")
+    src = tmp_path / "layout.c"
+    exe = tmp_path / "layout"
+    src.write_text("\n".join(lines))
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines():
+        cname, what, value = line.split()
+        got[(cname, what)] = int(value)
+    for cname, py in structs.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for field, _ in py._fields_:
+            assert got[(cname, field)] == getattr(py, field).offset, (cname, field)

@@ -275,3 +275,56 @@ def test_one_cta_and_pair_kernels_agree(lib, tmp_path):
     check(one, ref["y"], "one-CTA kernel")
     check(pair, ref["y"], "pair kernel")
     assert np.array_equal(one, pair)
+
+
+# ------------------------------------------------------------------------------------------
+# fused output amax (delayed scale of the next call's requant)
+# ------------------------------------------------------------------------------------------
+
+def bf16_absmax(t):
+    return float(t.float().abs().max().item())
+
+
+@pytest.mark.parametrize("M", [300, 129])
+def test_out_amax_equals_max_of_bf16_output(lib, M):
+    case = W.case_bias(M, 512, 768, seed=M, w_std=0.05)
+    amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+    aq = B.quantize(case.x.cuda())
+    wq = B.quantize(case.w.cuda())
+    out = B.linear(aq, wq, "bias", bias=case.bias.cuda(), out_amax=amax)
+    B.check_device_error()
+    assert float(amax.item()) == bf16_absmax(out)
+    _, _, ref = run_oracle(case)
+    assert abs(float(amax.item()) - float(np.max(np.abs(ref["y"])))) <= TOL * float(np.max(np.abs(ref["y"])))
+
+
+def test_out_amax_with_fp4_only_output(lib):
+    case = W.case_ffn_up(300, K=512, F=256, seed=8)
+    aq = B.quantize(case.x.cuda())
+    wq = B.quantize(case.w.cuda())
+    bf16_out = B.linear(aq, wq, "gated_silu")
+    q = B.QTensor.empty(300, 256)
+    q.g.fill_(bf16_absmax(bf16_out) / 2688.0)
+    amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+    B.linear(aq, wq, "gated_silu", out_fp4=q, want_bf16=False, out_amax=amax)
+    B.check_device_error()
+    assert float(amax.item()) == bf16_absmax(bf16_out)
+    # the delayed scale is the one the quantiser computes for the same output
+    q2 = B.quantize(bf16_out)
+    torch.cuda.synchronize()
+    assert float(q2.g.item()) == np.float32(np.float32(amax.item()) / np.float32(2688.0))
+
+
+def test_out_amax_ignores_rows_past_m(lib):
+    # x = 1 and w = -50/256 quantise to full-scale codes (block scale 448), so every real output is
+    # acc * alpha + bias = -50 + 50 up to the rounding of the fp32 tensor scales (|y| ~ 1e-5); the
+    # tile's rows past M (zero A rows) would read the bias alone, 50
+    M, N, K = 100, 256, 256
+    x = torch.ones(M, K, dtype=torch.bfloat16, device="cuda")
+    w = torch.full((N, K), -50.0 / 256.0, dtype=torch.bfloat16, device="cuda")
+    bias = torch.full((N,), 50.0, dtype=torch.bfloat16, device="cuda")
+    amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+    out = B.linear(B.quantize(x), B.quantize(w), "bias", bias=bias, out_amax=amax)
+    B.check_device_error()
+    assert bf16_absmax(out) < 1e-3
+    assert float(amax.item()) == bf16_absmax(out)
