@@ -432,7 +432,7 @@ def op_case(name):
     from epilogue_gemm_nvfp4_b200 import binding as B
     dev = torch.device("cuda")
 
-    def gemm(case, requant=False):
+    def gemm(case, requant=False, with_amax=False):
         a = B.quantize(case.x.to(dev))
         w = B.quantize(case.w.to(dev))
         bias = case.bias.to(dev) if case.bias is not None else None
@@ -448,6 +448,8 @@ def op_case(name):
             q = B.QTensor.empty(case.M, case.n_out)
             q.g.fill_(0.01)
         out = torch.empty(case.M, case.n_out, dtype=torch.bfloat16, device=dev)
+        if with_amax:  # the epilogue also publishes max |output| (the next call's delayed requant scale)
+            ex["out_amax"] = torch.zeros(1, dtype=torch.float32, device=dev)
         fn = lambda: B.linear(a, w, case.epilogue, bias=bias, out=out if q is None else None, out_fp4=q,
                               want_bf16=q is None, **ex)
         return fn, W.flops(case), "TFLOP/s"
@@ -457,6 +459,12 @@ def op_case(name):
         q = B.QTensor.empty(rows, cols)
         q.g.fill_(3.0 / 2688.0)
         return (lambda: B.quantize(x, out=q, static=static)), 2.5625 * rows * cols, "GB/s (2.5625 B/elem)"
+
+    def fakeq(rows, cols, static=False):
+        x = W.to_bf16(W.normal(np.random.default_rng(0), (rows, cols))).to(dev)
+        y = torch.empty(rows, cols, dtype=torch.bfloat16, device=dev)
+        scale = torch.full((1,), 3.0 / 2688.0, dtype=torch.float32, device=dev)
+        return (lambda: B.fake_quantize(x, y=y, scale=scale, static=static)), 4.0 * rows * cols, "GB/s (4 B/elem)"
 
     def amax(rows, cols):
         x = W.to_bf16(W.normal(np.random.default_rng(0), (rows, cols))).to(dev)
@@ -469,6 +477,7 @@ def op_case(name):
         "tiny": lambda: gemm(W.tiny()),
         "qkv_1k": lambda: gemm(W.qkv_1k()),
         "up_1k": lambda: gemm(W.case_ffn_up(M1), requant=True),
+        "up_1k_amax": lambda: gemm(W.case_ffn_up(M1), requant=True, with_amax=True),
         "down_1k": lambda: gemm(W.case_ffn_down(M1)),
         "text_512": lambda: gemm(W.text_proj(W.PROMPT_T)),
         "text_1941": lambda: gemm(W.text_proj(W.LONG_PROMPT_T)),
@@ -478,6 +487,8 @@ def op_case(name):
         "quant_2k": lambda: quant(M2, W.HIDDEN),
         "quant_text": lambda: quant(W.HIDDEN, W.TEXT_K),
         "quant_2k_static": lambda: quant(M2, W.HIDDEN, static=True),
+        "fakeq_2k": lambda: fakeq(M2, W.HIDDEN),
+        "fakeq_2k_static": lambda: fakeq(M2, W.HIDDEN, static=True),
         "quant_text_static": lambda: quant(W.HIDDEN, W.TEXT_K, static=True),
         "amax_2k": lambda: amax(M2, W.HIDDEN),
     }

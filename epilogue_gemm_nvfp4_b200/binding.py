@@ -19,7 +19,8 @@ LIB_PATH = os.path.join(_HERE, "libnvfp4.so")
 #: every function the header declares
 EXPORTS = ("nvfp4_quantize", "nvfp4_linear", "nvfp4_dequantize", "nvfp4_amax", "nvfp4_scale_bytes",
            "nvfp4_scale_offset", "nvfp4_get_device_error", "nvfp4_linear_tile_n", "nvfp4_linear_split_k",
-           "nvfp4_status_string", "nvfp4_version", "nvfp4_linear_noalloc", "nvfp4_linear_noalloc_scratch_bytes")
+           "nvfp4_status_string", "nvfp4_version", "nvfp4_linear_noalloc", "nvfp4_linear_noalloc_scratch_bytes",
+           "nvfp4_fake_quantize")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_MISALIGNED, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_SCRATCH_LIMIT = range(7)
 EPI_BIAS, EPI_QKNORM, EPI_GATED_SILU, EPI_RESID_GATE = range(4)
@@ -65,6 +66,7 @@ def load() -> ctypes.CDLL:
         "nvfp4_linear_noalloc": (I32, [TP, TP, EP, P, I64, TP, P]),
         "nvfp4_linear_noalloc_scratch_bytes": (SZ, []),
         "nvfp4_dequantize": (I32, [TP, P, I64, P]),
+        "nvfp4_fake_quantize": (I32, [P, I64, I64, I64, I32, P, P, I64, P]),
         "nvfp4_amax": (I32, [P, I64, I64, I64, P, P]),
         "nvfp4_scale_bytes": (SZ, [I64, I64]),
         "nvfp4_scale_offset": (I64, [I64, I64, I64]),
@@ -156,6 +158,24 @@ def quantize(x: torch.Tensor, out: QTensor | None = None, g: float | torch.Tenso
     _check(load().nvfp4_quantize(_ptr(x), rows, cols, x.stride(0), int(compute), ctypes.byref(ct),
                                  _stream(stream)), "nvfp4_quantize")
     return out
+
+
+def fake_quantize(x: torch.Tensor, y: torch.Tensor | None = None, g: float | torch.Tensor | None = None,
+                  scale: torch.Tensor | None = None, static: bool = False,
+                  stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """y = dequantize(quantize(x)) in bf16, one pass.  By default g is computed on the device and
+    returned in ``scale`` (one fp32 element); with ``g`` the given decode scale is stored there and
+    used; with ``static=True`` the value already in ``scale`` is used."""
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    y = torch.empty((rows, cols), dtype=torch.bfloat16, device=x.device) if y is None else y
+    scale = torch.empty(1, dtype=torch.float32, device=x.device) if scale is None else scale
+    if g is not None:
+        scale.copy_(torch.as_tensor(g, dtype=torch.float32).reshape(1))
+    compute = g is None and not static
+    _check(load().nvfp4_fake_quantize(_ptr(x), rows, cols, x.stride(0), int(compute), _ptr(scale), _ptr(y),
+                                      y.stride(0), _stream(stream)), "nvfp4_fake_quantize")
+    return y, scale
 
 
 def dequantize(q: QTensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:

@@ -370,6 +370,35 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
   return launch_status();
 }
 
+nvfp4_status nvfp4_fake_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int32_t compute_scale,
+                                 float* tensor_scale, void* y, int64_t ldy, nvfp4_stream_t stream) {
+  if (!x || !y || !tensor_scale || rows < 0 || cols <= 0 || ldx < cols || ldy < cols) return NVFP4_ERR_INVALID_ARG;
+  if (cols % 16) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || (ldx * 2) % 16 || !aligned16(y) || (ldy * 2) % 16 || !aligned4(tensor_scale))
+    return NVFP4_ERR_MISALIGNED;
+  DeviceState* st;
+  if (nvfp4_status e = device_state(&st)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  const int64_t steps = (cols / 16 + 31) / 32;
+  const int64_t tasks = rows * ((steps + kQuantStepsPerTask - 1) / kQuantStepsPerTask) + 1;
+  const bool vec32 = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx * 2) % 32 == 0;
+  // as in nvfp4_quantize: after the amax pass, walk the tensor back to front
+  auto fk = compute_scale ? (vec32 ? fake_quantize_kernel<true, true> : fake_quantize_kernel<true, false>)
+                          : (vec32 ? fake_quantize_kernel<false, true> : fake_quantize_kernel<false, false>);
+  if (compute_scale) {
+    unsigned int* state = nullptr;
+    if (nvfp4_status e = amax_state_for(s, &state)) return e;
+    const int agrid = resident_grid(amax_scale_kernel, 256, rows * cols / 8, 256 * 4, st->sm_count);
+    amax_scale_kernel<<<agrid, 256, 0, s>>>(xb, rows, cols, ldx, state, tensor_scale);
+  }
+  if (rows > 0) {
+    const int grid = resident_grid(fk, 256, tasks, 8, st->sm_count);
+    fk<<<grid, 256, 0, s>>>(xb, rows, cols, ldx, tensor_scale, static_cast<__nv_bfloat16*>(y), ldy);
+  }
+  return launch_status();
+}
+
 nvfp4_status nvfp4_dequantize(const nvfp4_tensor* t, void* out_bf16, int64_t ld_out, nvfp4_stream_t stream) {
   if (!out_bf16) return NVFP4_ERR_INVALID_ARG;
   if (nvfp4_status e = check_tensor(t, true, 8)) return e;

@@ -221,6 +221,84 @@ __global__ void __launch_bounds__(256, 6) quantize_kernel(const __nv_bfloat16* _
 // dequantise: one thread per 16-element block.
 // ------------------------------------------------------------------------------------------
 
+// ------------------------------------------------------------------------------------------
+// fake quantisation: y = dequantise(quantise(x, g)) in bf16, one pass, no codes kept (the forward of
+// quantisation-aware training).  Per block: the quantiser's block rule and codes, then the
+// dequantiser's decode (e2m1(code) * (e4m3(s) * g), each product in fp32, then bf16 RNE), so y equals
+// nvfp4_quantize followed by nvfp4_dequantize bit for bit.  Same task layout as quantize_kernel.
+// ------------------------------------------------------------------------------------------
+
+template <bool kReverse, bool kVec32>
+__global__ void __launch_bounds__(256, 6) fake_quantize_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
+                                                            int64_t cols, int64_t ldx,
+                                                            const float* __restrict__ scale_src,
+                                                            __nv_bfloat16* __restrict__ y, int64_t ldy) {
+  const float g = *scale_src;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t gwarp = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int bpr = static_cast<int>(cols / 16);
+  const int steps = (bpr + 31) / 32;
+  const int chunks = (steps + kQuantStepsPerTask - 1) / kQuantStepsPerTask;
+  const int per_chunk = (steps + chunks - 1) / chunks;
+  const int64_t total = rows * chunks;
+
+  for (int64_t t = gwarp; t < total; t += nwarps) {
+    const int64_t tt = kReverse ? total - 1 - t : t;
+    const int64_t row = tt / chunks;
+    const int chunk = static_cast<int>(tt - row * chunks);
+    const int st_begin = chunk * per_chunk;
+    const int st_end = min(steps, st_begin + per_chunk);
+    const __nv_bfloat16* xrow = x + row * ldx;
+    __nv_bfloat16* yrow = y + row * ldy;
+    for (int st = st_begin; st < st_end; st += kQuantUnroll) {
+      uint32_t w[kQuantUnroll][8];
+#pragma unroll
+      for (int u = 0; u < kQuantUnroll; ++u) {
+        const int blk = (st + u) * 32 + lane;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[u][i] = 0;
+        if (st + u < st_end && blk < bpr) ld_block32(xrow + blk * 16, kVec32, w[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < kQuantUnroll; ++u) {
+        if (st + u >= st_end) break;  // warp-uniform
+        const int blk = (st + u) * 32 + lane;
+        if (blk >= bpr) continue;
+        uint32_t m2 = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m2 = __vmaxu2(m2, w[u][i] & 0x7FFF7FFFu);
+        const uint32_t mb = max(m2 & 0xFFFFu, m2 >> 16);
+        float inv;
+        const uint32_t sc = block_scale(__uint_as_float(mb << 16), g, inv);
+        const float d = __fmul_rn(e4m3_to_float(sc), g);
+        uint32_t o[8];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float q[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            q[2 * i] = __fmul_rn(__uint_as_float(w[u][4 * h + i] << 16), inv);
+            q[2 * i + 1] = __fmul_rn(__uint_as_float(w[u][4 * h + i] & 0xFFFF0000u), inv);
+          }
+          const uint32_t codes8 = (inv == 0.0f) ? 0u : e2m1x8(q);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t byte = (codes8 >> (8 * i)) & 0xFFu;
+            const __nv_bfloat16 lo = __float2bfloat16_rn(__fmul_rn(e2m1_to_float(byte & 0xFu), d));
+            const __nv_bfloat16 hi = __float2bfloat16_rn(__fmul_rn(e2m1_to_float(byte >> 4), d));
+            o[4 * h + i] = static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
+                           (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+          }
+        }
+        uint4* dst = reinterpret_cast<uint4*>(yrow + blk * 16);
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restrict__ codes, int64_t ld_codes,
                                                          const uint8_t* __restrict__ scales,
                                                          const float* __restrict__ gptr, int64_t rows, int64_t cols,

@@ -179,6 +179,21 @@ NVFP4_API nvfp4_status nvfp4_linear_noalloc(const nvfp4_tensor* a, const nvfp4_t
 /* Size in bytes of the fixed split-K scratch array used by nvfp4_linear_noalloc. */
 NVFP4_API size_t nvfp4_linear_noalloc_scratch_bytes(void);
 
+/*
+ * Fake quantisation (the forward of quantisation-aware training): y = dequantise(quantise(x)) as bf16
+ * [rows, ldy], in one pass that keeps no codes.  y equals nvfp4_quantize followed by nvfp4_dequantize
+ * with the same scale, bit for bit.
+ *   compute_scale = 1: g = amax(|x|) / 2688 (1 for an all-zero or empty x) is computed on the device
+ *                      and written to *tensor_scale (the amax pass of nvfp4_quantize, with the same
+ *                      per-stream state and the same rule on graph capture).
+ *   compute_scale = 0: *tensor_scale holds g.
+ * Rules: cols % 16 == 0; x, y, ldx*2 and ldy*2 16-byte aligned; ldy >= cols; tensor_scale 4-byte
+ * aligned.  rows == 0 writes nothing to y.
+ */
+NVFP4_API nvfp4_status nvfp4_fake_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx,
+                                           int32_t compute_scale, float* tensor_scale, void* y, int64_t ldy,
+                                           nvfp4_stream_t stream);
+
 /* Dequantise t to bf16 [t->rows, ld_out]: value = e2m1(code) * (e4m3(scale) * g), each product in fp32
  * rounded to nearest even, then rounded to bf16.  Rules as for nvfp4_quantize. */
 NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor* t, void* out_bf16, int64_t ld_out, nvfp4_stream_t stream);

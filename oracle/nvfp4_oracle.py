@@ -186,6 +186,16 @@ def dequantize(codes: np.ndarray, scales: np.ndarray, g) -> np.ndarray:
     return (vals * d[:, :, None]).astype(F32).reshape(M, K)
 
 
+def fake_quantize(x: np.ndarray, g: np.float32 | None = None):
+    """The forward value of training through the quantiser's own noise ("Serving sub-second Ideogram v4
+    without quality loss", the passage on quantization-aware distillation: the student learns through
+    its 4-bit rounding with a straight-through estimator, whose forward is the quantised value).  That
+    value is the NVFP4 round trip: the block rule, then e2m1(code) * d, rounded to bf16.
+    x float32 [M,K] (bf16 values) -> (y float32 of bf16 values [M,K], g)."""
+    codes, scales, g = quantize(x, g)
+    return to_bf16_round(dequantize(codes, scales, g)), g
+
+
 def dequantize_exact(codes: np.ndarray, scales: np.ndarray, g) -> np.ndarray:
     """fp64 e2m1(code) * float(s) * g, exact (3 + 4 + 24 significant bits fit in 53)."""
     M, K = codes.shape

@@ -107,3 +107,32 @@ def test_dynamic_scale_state_is_per_call_and_per_stream(lib):
     side.synchronize()
     assert_quant_bitexact(q, ref[id(small)], 300, 512)
     assert_quant_bitexact(B.quantize(big.cuda()), ref[id(big)], 300, 512)
+
+
+# ------------------------------------------------------------------------------------------
+# fake quantisation: y = dequantise(quantise(x)) in one pass
+# ------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("rows,cols,seed", [(1, 16, 0), (130, 208, 2), (300, 4608, 5), (33, 53248, 6)])
+def test_fake_quantize_bitexact(lib, rows, cols, seed):
+    x = rand_bf16(rows, cols, seed, dist="t" if seed % 2 else "normal")
+    y, g = B.fake_quantize(x.cuda())
+    ref_y, ref_g = O.fake_quantize(f32(x))
+    torch.cuda.synchronize()
+    assert float(g.item()) == float(ref_g)
+    np.testing.assert_array_equal(f32(y), ref_y)
+    # and it equals the library's own quantise followed by dequantise
+    q = B.quantize(x.cuda())
+    np.testing.assert_array_equal(f32(y), f32(B.dequantize(q)))
+
+
+def test_fake_quantize_static_scale_and_strides(lib):
+    base = rand_bf16(96, 512 + 64, 17)
+    x = base.cuda()[:, 32:32 + 512]             # row stride 576 elements, 64-byte offset
+    y = torch.empty(96, 512 + 16, dtype=torch.bfloat16, device="cuda")[:, :512]
+    g = 0.7 / 2688.0
+    out, scale = B.fake_quantize(x, y=y, g=g)
+    torch.cuda.synchronize()
+    assert out.data_ptr() == y.data_ptr()
+    ref_y, _ = O.fake_quantize(f32(base)[:, 32:32 + 512], np.float32(g))
+    np.testing.assert_array_equal(f32(out), ref_y)

@@ -373,3 +373,42 @@ def test_page_sizes_pin_workload_shapes():
     assert 2 * W.IMG_TOKENS_1K * W.TEXT_K * 2 / 2 ** 30 == p["zero_rows_saving_1k"][0]
     assert 2 * W.IMG_TOKENS_2K * W.TEXT_K * 2 / 2 ** 30 == p["zero_rows_saving_2k"][0]
     assert W.N_HEADS * W.HEAD_DIM == W.HIDDEN
+
+
+# ------------------------------------------------------------------------------------------
+# fake quantisation (the forward of training through the quantiser's noise)
+# ------------------------------------------------------------------------------------------
+
+def test_fake_quantize_leaves_grid_values_unchanged():
+    """Blocks already on the NVFP4 grid (e2m1 codes times one E4M3 value, with a full-scale code in each
+    block, tensor scale 1) come back exactly: the round trip's fixed points, by the format's definition."""
+    rng = np.random.default_rng(23)
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], dtype=np.float64)
+    block_scales = np.array([0.25, 0.5, 1.0, 2.0, 8.0, 16.0])  # exact E4M3 values, 6 * s exact in bf16
+    M, K = 8, 64
+    x = np.empty((M, K))
+    for r in range(M):
+        for b in range(K // 16):
+            v = grid[rng.integers(0, 8, 16)] * rng.choice([-1.0, 1.0], 16)
+            v[rng.integers(0, 16)] = 6.0 * rng.choice([-1.0, 1.0])  # the block's amax is 6 * s
+            x[r, 16 * b:16 * b + 16] = v * block_scales[(r + b) % len(block_scales)]
+    x = x.astype(np.float32)
+    y, g = O.fake_quantize(x, np.float32(1.0))
+    assert g == np.float32(1.0)
+    np.testing.assert_array_equal(y, x)
+
+
+def test_fake_quantize_element_rounding_matches_ml_dtypes():
+    """Each element is the ml_dtypes E2M1 rounding of x * inv, times d, rounded to bf16: an independent
+    statement of the element step, with the block scale from the oracle's own quantiser."""
+    rng = np.random.default_rng(29)
+    x = (rng.standard_normal((16, 128)) * 3).astype(ml_dtypes.bfloat16).astype(np.float32)
+    y, g = O.fake_quantize(x)
+    _, scales, _ = O.quantize(x, g)
+    d = (O.e4m3_decode(scales).astype(np.float32) * np.float32(g)).astype(np.float32)
+    d = np.repeat(d, 16, axis=1)
+    inv = np.where(d == 0, np.float32(0), (np.float32(1) / np.where(d == 0, np.float32(1), d)).astype(np.float32))
+    v = (x * inv).astype(np.float32)
+    e = v.astype(ml_dtypes.float4_e2m1fn).astype(np.float32)
+    ref = (e * d).astype(np.float32).astype(ml_dtypes.bfloat16).astype(np.float32)
+    np.testing.assert_array_equal(y, ref)
