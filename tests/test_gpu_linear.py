@@ -328,3 +328,41 @@ def test_out_amax_ignores_rows_past_m(lib):
     B.check_device_error()
     assert bf16_absmax(out) < 1e-3
     assert float(amax.item()) == bf16_absmax(out)
+
+
+def test_cuda_graph_capture_and_replay(lib):
+    """Dynamic-scale quantise + fused linear captured in a CUDA graph replays to the eager bits.  The
+    first dynamic quantise on a stream allocates that stream's reduction state, so it runs eagerly on
+    the capture stream before the capture."""
+    case = W.case_qkv(300, n_heads=2, K=512, seed=12)
+    x = case.x.cuda()
+    wq = B.quantize(case.w.cuda())
+    bias = case.bias.cuda()
+    aq = B.QTensor.empty(300, 512)
+    out = torch.empty(300, case.n_out, dtype=torch.bfloat16, device="cuda")
+    amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+    epi = gpu_epi_kwargs(case)
+
+    def run():
+        B.quantize(x, out=aq)
+        B.linear(aq, wq, "qknorm", bias=bias, out=out, out_amax=amax, **epi)
+
+    cs = torch.cuda.Stream()
+    with torch.cuda.stream(cs):
+        run()
+    cs.synchronize()
+    B.check_device_error()
+    eager, eager_codes, eager_g = out.clone(), aq.codes.clone(), aq.g.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=cs):
+        run()
+    for _ in range(2):
+        out.zero_()
+        aq.codes.zero_()
+        amax.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager)
+        assert torch.equal(aq.codes, eager_codes) and torch.equal(aq.g, eager_g)
+        assert float(amax.item()) == bf16_absmax(eager)
+    B.check_device_error()
