@@ -17,7 +17,8 @@
 //   warps 4-7  scale stagers into this CTA's TMEM, then an arrival on the leader's `full`.
 //   warps 8-15 epilogue of this CTA's 128 rows; the accumulator release is an arrival on the
 //              leader's `acc_empty` (16 arrivals: 8 warps per CTA).
-// Split-K and 128-wide tiles stay on the one-CTA kernel.
+// 128-wide tiles stay on the one-CTA kernel.  Split-K units exchange partial sums per (pair tile,
+// rank) exactly as the one-CTA kernel does per tile.
 #pragma once
 
 #include "gemm.cuh"
@@ -62,17 +63,25 @@ struct GemmPairCfg {
 };
 
 struct PairUnit {
-  int mp, nb;  // 256-row block pair, 256-wide B block
+  int tile, mp, nb;  // pair tile = 256-row block pair x 256-wide B block
+  int kb0, kb1;      // this unit's range of stages along K (split-K)
 };
 
-__device__ __forceinline__ PairUnit pair_unit(const GemmArgs& a, int u) {
+// As in the one-CTA kernel, the `splits` units of one tile are adjacent in the grid-stride order, so
+// they run in the same wave on neighbouring clusters.
+__device__ __forceinline__ PairUnit pair_unit(const GemmArgs& a, int u, int num_kb) {
   PairUnit w;
-  w.mp = u % a.num_m_pairs;
-  w.nb = u / a.num_m_pairs;
+  const int split = u % a.splits;
+  w.tile = u / a.splits;
+  w.mp = w.tile % a.num_m_pairs;
+  w.nb = w.tile / a.num_m_pairs;
+  w.kb0 = split * num_kb / a.splits;
+  w.kb1 = (split + 1) * num_kb / a.splits;
   return w;
 }
 
-template <int KIND>
+// kSplit: the instantiation with the split-K exchange (the host uses it when splits > 1)
+template <int KIND, bool kSplit>
 __global__ void __launch_bounds__(512, 1) __cluster_dims__(2, 1, 1)
     nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                            const __grid_constant__ OutMaps out_maps, const __grid_constant__ GemmArgs args) {
@@ -88,6 +97,7 @@ __global__ void __launch_bounds__(512, 1) __cluster_dims__(2, 1, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* never_abort = abort_flag + 1;
+  volatile int* split_role = never_abort + 1;
   float* ss_x = reinterpret_cast<float*>(smem_raw + C::SS_OFFSET);
   uint8_t* ring = smem_raw + C::AUX_BYTES;
   ring += (1024u - (smem_u32(ring) & 1023u)) & 1023u;
@@ -142,10 +152,10 @@ __global__ void __launch_bounds__(512, 1) __cluster_dims__(2, 1, 1)
         uint32_t armed_mask = 0, armed_parity = 0;
         bool ok = true;
         for (int u = cluster; ok && u < args.num_units; u += num_clusters) {
-          const PairUnit pu = pair_unit(args, u);
+          const PairUnit pu = pair_unit(args, u, num_kb);
           const int mb = 2 * pu.mp + static_cast<int>(rank);  // this CTA's 128-row block of A
           const bool a_rows = mb < args.num_m_blocks;         // false: the block lies wholly past M
-          for (int kb = 0; kb < num_kb; ++kb) {
+          for (int kb = pu.kb0; kb < pu.kb1; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.timeout_ns)) {
               ok = false;
               break;
@@ -201,13 +211,14 @@ __global__ void __launch_bounds__(512, 1) __cluster_dims__(2, 1, 1)
         uint32_t aphase = 0;
         bool ok = true;
         for (int u = cluster; ok && u < args.num_units; u += num_clusters) {
+          const PairUnit pu = pair_unit(args, u, num_kb);
           if (!mbar_wait(&acc_empty[0], aphase ^ 1u, abort_flag, args.timeout_ns)) {
             ok = false;
             break;
           }
           tc_fence_after();
           uint32_t accumulate = 0;
-          for (int kb = 0; kb < num_kb; ++kb) {
+          for (int kb = pu.kb0; kb < pu.kb1; ++kb) {
             if (!mbar_wait(&full[stage], phase, abort_flag, args.timeout_ns)) {
               ok = false;
               break;
@@ -257,9 +268,9 @@ __global__ void __launch_bounds__(512, 1) __cluster_dims__(2, 1, 1)
     uint32_t phase = 0;
     bool ok = true;
     for (int u = cluster; ok && u < args.num_units; u += num_clusters) {
-      const PairUnit pu = pair_unit(args, u);
+      const PairUnit pu = pair_unit(args, u, num_kb);
       const bool a_rows = 2 * pu.mp + static_cast<int>(rank) < args.num_m_blocks;
-      for (int kb = 0; kb < num_kb; ++kb) {
+      for (int kb = pu.kb0; kb < pu.kb1; ++kb) {
         const bool got = mbar_wait(&sf_landed[stage], phase, abort_flag, args.timeout_ns);
         if (!__all_sync(0xFFFFFFFFu, got)) {
           ok = false;
@@ -319,7 +330,7 @@ __global__ void __launch_bounds__(512, 1) __cluster_dims__(2, 1, 1)
     uint32_t aphase = 0;
     uint32_t amax_bits = 0;
     for (int u = cluster; u < args.num_units; u += num_clusters) {
-      const PairUnit pu = pair_unit(args, u);
+      const PairUnit pu = pair_unit(args, u, num_kb);
       const int mb = 2 * pu.mp + static_cast<int>(rank);
       const int nb = pu.nb;
       const __nv_bfloat16* gamma = nullptr;
@@ -342,6 +353,13 @@ __global__ void __launch_bounds__(512, 1) __cluster_dims__(2, 1, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_acc_empty);
       aphase ^= 1u;
+      // split-K: the unit that finishes first parks its partial sums and moves on; the second adds
+      // them and runs the epilogue (exchange slot = this CTA's half of the pair tile)
+      if constexpr (kSplit && KIND != kEpiQkNorm) {
+        if (!split_exchange<E::COLS>(args, 2 * pu.tile + static_cast<int>(rank), e, q * 32 + lane, acc,
+                                     split_role, abort_flag))
+          continue;
+      }
       float ss = 0.0f;
       if (KIND == kEpiQkNorm && gamma != nullptr) ss = E::head_sumsq(args, e, nb, q * 32 + lane, alpha, acc, ss_x);
       E::finish(args, &out_maps, xpose, row0, row0 + lane, e, nb, alpha, qg, gamma, ss, acc, amax_bits);

@@ -28,7 +28,7 @@ struct DeviceState {
   int sm_count = 0;
   unsigned int* error_word = nullptr;
   bool smem_attr_set[2][4] = {};
-  int pair_clusters[4] = {};  // resident CTA pairs per epilogue kind (0 until first use)
+  int pair_clusters[2][4] = {};  // resident CTA pairs per (split-K, epilogue kind), 0 until first use
 };
 
 std::mutex g_mutex;
@@ -251,12 +251,12 @@ bool pair_kernel_enabled() {
   return on;
 }
 
-template <int KIND>
-nvfp4_status launch_gemm_pair(DeviceState* st, const CUtensorMap& ma, const CUtensorMap& mb, const OutMaps& om,
-                              const GemmArgs& args, cudaStream_t stream) {
+template <int KIND, bool kSplit>
+nvfp4_status launch_gemm_pair_as(DeviceState* st, const CUtensorMap& ma, const CUtensorMap& mb, const OutMaps& om,
+                                 const GemmArgs& args, cudaStream_t stream) {
   using C = GemmPairCfg;
-  auto kernel = nvfp4_gemm_pair_kernel<KIND>;
-  int& clusters = st->pair_clusters[KIND];
+  auto kernel = nvfp4_gemm_pair_kernel<KIND, kSplit>;
+  int& clusters = st->pair_clusters[kSplit ? 1 : 0][KIND];
   if (clusters == 0) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
       return NVFP4_ERR_CUDA;
@@ -272,6 +272,17 @@ nvfp4_status launch_gemm_pair(DeviceState* st, const CUtensorMap& ma, const CUte
   const int grid_clusters = args.num_units < clusters ? args.num_units : clusters;
   kernel<<<2 * grid_clusters, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, om, args);
   return launch_status();
+}
+
+template <int KIND>
+nvfp4_status launch_gemm_pair(DeviceState* st, const CUtensorMap& ma, const CUtensorMap& mb, const OutMaps& om,
+                              const GemmArgs& args, cudaStream_t stream) {
+  if constexpr (KIND == kEpiQkNorm) {
+    return launch_gemm_pair_as<KIND, false>(st, ma, mb, om, args, stream);  // never split
+  } else {
+    return args.splits > 1 ? launch_gemm_pair_as<KIND, true>(st, ma, mb, om, args, stream)
+                           : launch_gemm_pair_as<KIND, false>(st, ma, mb, om, args, stream);
+  }
 }
 
 template <int BN, int KIND>
@@ -463,7 +474,7 @@ nvfp4_status linear_impl(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvf
   CUtensorMap ma, mb;
   if (nvfp4_status e = make_code_map(&ma, a)) return e;
   if (nvfp4_status e = make_code_map(&mb, w)) return e;
-  const bool pair = BN == 256 && split_k_for(K, epi->kind) == 1 && pair_kernel_enabled();
+  const bool pair = BN == 256 && pair_kernel_enabled();
   OutMaps om;
   if (nvfp4_status e = make_store_maps(&om, out_bf16, ld_out, epi->out_nvfp4 ? out_fp4 : nullptr, M, n_out,
                                        pair ? GemmPairCfg::XPOSE_BYTES / 64 : 16))
@@ -506,13 +517,16 @@ nvfp4_status linear_impl(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvf
   g.error_word = st->error_word;
   g.timeout_ns = wait_timeout_ns();
   g.splits = split_k_for(K, epi->kind);
+  if (pair) g.num_tiles = g.num_m_pairs * g.num_n_blocks;  // 256 x 256 tiles of CTA pairs
   g.num_units = g.num_tiles * g.splits;
+  // split-K exchange slots: one per tile, or one per CTA of each pair tile
+  const int64_t exch_slots = static_cast<int64_t>(g.num_tiles) * (pair ? 2 : 1);
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (g.splits > 1) {
     const int cols_per_thread = epi->kind == NVFP4_EPI_GATED_SILU ? 128 : BN / 2;
-    const size_t flag_bytes = (static_cast<size_t>(g.num_tiles) * 4 + 255) & ~size_t(255);
-    const size_t part_bytes = static_cast<size_t>(g.num_tiles) * 2 * 128 * cols_per_thread * 4;
+    const size_t flag_bytes = (static_cast<size_t>(exch_slots) * 4 + 255) & ~size_t(255);
+    const size_t part_bytes = static_cast<size_t>(exch_slots) * 2 * 128 * cols_per_thread * 4;
     void* ws = nullptr;
     if (fixed_scratch) {
       if (flag_bytes + part_bytes > kNoAllocScratchBytes) return NVFP4_ERR_SCRATCH_LIMIT;
@@ -522,11 +536,9 @@ nvfp4_status linear_impl(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvf
     }
     g.split_flags = static_cast<unsigned int*>(ws);
     g.split_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + flag_bytes);
-    if (cudaMemsetAsync(ws, 0, static_cast<size_t>(g.num_tiles) * 4, s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, static_cast<size_t>(exch_slots) * 4, s) != cudaSuccess) return NVFP4_ERR_CUDA;
   }
   if (pair) {
-    g.num_tiles = g.num_m_pairs * g.num_n_blocks;
-    g.num_units = g.num_tiles;
     switch (epi->kind) {
       case NVFP4_EPI_BIAS: return launch_gemm_pair<kEpiBias>(st, ma, mb, om, g, s);
       case NVFP4_EPI_RESID_GATE: return launch_gemm_pair<kEpiResidGate>(st, ma, mb, om, g, s);
