@@ -256,18 +256,24 @@ nvfp4_status launch_gemm_pair_as(DeviceState* st, const CUtensorMap& ma, const C
                                  const GemmArgs& args, cudaStream_t stream) {
   using C = GemmPairCfg;
   auto kernel = nvfp4_gemm_pair_kernel<KIND, kSplit>;
-  int& clusters = st->pair_clusters[kSplit ? 1 : 0][KIND];
-  if (clusters == 0) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    // clusters that can be resident at once: the persistent grid must not exceed one wave
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * (st->sm_count / 2));
-    cfg.blockDim = dim3(C::THREADS);
-    cfg.dynamicSmemBytes = C::SMEM_BYTES;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n < 1) return NVFP4_ERR_CUDA;
-    clusters = n;
+  int clusters = 0;
+  {
+    // first use on this device (under the library lock, so concurrent callers do it once)
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int& cached = st->pair_clusters[kSplit ? 1 : 0][KIND];
+    if (cached == 0) {
+      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+      // clusters that can be resident at once: the persistent grid must not exceed one wave
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (st->sm_count / 2));
+      cfg.blockDim = dim3(C::THREADS);
+      cfg.dynamicSmemBytes = C::SMEM_BYTES;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n < 1) return NVFP4_ERR_CUDA;
+      cached = n;
+    }
+    clusters = cached;
   }
   const int grid_clusters = args.num_units < clusters ? args.num_units : clusters;
   kernel<<<2 * grid_clusters, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, om, args);
@@ -290,11 +296,14 @@ nvfp4_status launch_gemm(DeviceState* st, const CUtensorMap& ma, const CUtensorM
                          const GemmArgs& args, cudaStream_t stream) {
   using C = GemmCfg<BN>;
   auto kernel = nvfp4_gemm_kernel<BN, KIND>;
-  bool& attr = st->smem_attr_set[BN == 256 ? 1 : 0][KIND];
-  if (!attr) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    attr = true;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    bool& attr = st->smem_attr_set[BN == 256 ? 1 : 0][KIND];
+    if (!attr) {
+      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+      attr = true;
+    }
   }
   const int grid = args.num_units < st->sm_count ? args.num_units : st->sm_count;
   kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, om, args);
