@@ -304,7 +304,7 @@ def run_native(args, ws, rank, local):
     host_out = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in bs.out.items()}
     h2d = sum(t.numel() * t.element_size() for t in host_in.values()) + host_res.numel() * host_res.element_size()
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-    e2e_steps = max(4, min(args.steps, 10))
+    e2e_steps = max(4, min(args.steps, 20))
     slots = [bs, bs.io_slot()]
     s_in, s_c, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
