@@ -149,6 +149,11 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols,
  * Rules: K % 64 == 0, K >= 64; N % 128 == 0 (N % 256 == 0 for QKNORM and GATED_SILU); M >= 1 (any);
  * all pointers and ld_out * 2 16-byte aligned.  The per-row arithmetic does not depend on M: row m of
  * the output is bitwise the same whatever rows accompany it.
+ * Kernels: 256-wide tiles (N % 256 == 0) run on two-CTA clusters with the paired tensor-core MMA;
+ * other tiles on single CTAs.  The environment variable NVFP4_GEMM_PAIR=0, read once per process,
+ * keeps every tile on single CTAs; the results are the same bits.  K >= 32768 splits the reduction
+ * in two halves summed in a fixed order, using per-stream scratch that the library allocates on
+ * first use (nvfp4_linear_noalloc uses a fixed array instead).
  */
 NVFP4_API nvfp4_status nvfp4_linear(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvfp4_epilogue_desc* epi,
                           void* out_bf16, int64_t ld_out, const nvfp4_tensor* out_fp4, nvfp4_stream_t stream);

@@ -88,6 +88,20 @@ def test_argument_checks_return_before_any_launch(lib):
     assert lib.nvfp4_quantize(0x10000, 5, 512, 512, 1, ctypes.byref(t), None) == B.ERR_INVALID_ARG
     assert lib.nvfp4_dequantize(ctypes.byref(t), None, 512, None) == B.ERR_INVALID_ARG
     assert lib.nvfp4_amax(0x10000, 4, 512, 512, None, None) == B.ERR_INVALID_ARG
+    # fused output amax: a 4-byte aligned fp32 slot
+    am = B.CEpilogue(out_amax=0x10002)
+    assert lin(a, w, am) == B.ERR_MISALIGNED
+    # fake quantisation
+    fq = lambda x=0x10000, rows=4, cols=512, ldx=512, cs=1, g=0x10000, y=0x10000, ldy=512: \
+        lib.nvfp4_fake_quantize(x, rows, cols, ldx, cs, g, y, ldy, None)
+    assert fq(x=None) == B.ERR_INVALID_ARG
+    assert fq(y=None) == B.ERR_INVALID_ARG
+    assert fq(g=None) == B.ERR_INVALID_ARG
+    assert fq(cols=520, ldx=520, ldy=520) == B.ERR_UNSUPPORTED_SHAPE                     # cols % 16
+    assert fq(ldy=256) == B.ERR_INVALID_ARG                                                 # ldy < cols
+    assert fq(y=0x10008) == B.ERR_MISALIGNED
+    assert fq(ldx=516) == B.ERR_MISALIGNED
+    assert fq(g=0x10001) == B.ERR_MISALIGNED
 
 
 @pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-device path")
