@@ -125,7 +125,7 @@ __device__ __forceinline__ uint32_t block_scale(float amax_b, float g, float& in
 // re-read from L2 what that pass left there.
 // ------------------------------------------------------------------------------------------
 
-constexpr int kQuantStepsPerTask = 8;   // 8 x 512 elements of one row per warp task
+constexpr int kQuantStepsPerTask = 16;  // up to 16 x 512 elements of one row per warp task
 constexpr int kQuantUnroll = 2;         // 32-byte loads in flight per lane
 
 __device__ __forceinline__ void ld_block32(const __nv_bfloat16* p, bool vec32, uint32_t (&w)[8]) {
