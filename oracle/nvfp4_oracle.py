@@ -324,6 +324,49 @@ def linear(a_q, w_q, kind="bias", bias=None, rows=None, out_g=None, **ex):
     return out
 
 
+# ---------------------------------------------------------------------------------------------
+# adaLN prologue of the quantiser (fp64, then one bf16 rounding)
+# ---------------------------------------------------------------------------------------------
+
+def adaln_modulate(x, shift=None, scale=None, eps: float = 1e-6, rows_per_sample: int = 0):
+    """The op in front of a DiT block's QKV and FFN-up products, as the plain definition in fp64.
+
+    "Serving sub-second Ideogram v4 without quality loss" (paragraph on kernel fusion) names RMSNorm
+    as one of the small ops that chase the big products, and "Quantizing a Dual-Branch Flow-Matching
+    Diffusion Transformer for Consumer GPUs" (related-work paragraph on W8A8) names adaLN's
+    modulation, generated at run time, as what the hidden state goes through before a linear.
+    Neither page writes the formula; the reading is the usual adaLN form on an RMS-normalised row:
+
+        rstd[r] = 1 / sqrt(mean_k x[r,k]^2 + eps)
+        u[r,k]  = x[r,k] * rstd[r] * (1 + scale[b,k]) + shift[b,k],   b = r // rows_per_sample
+
+    (b = 0 for every row when rows_per_sample is 0).  shift / scale are [S, C] (or [C]); None means
+    zeros.  Returns (u fp64 [M, C], rstd fp64 [M]).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    M, C = x.shape
+    rstd = 1.0 / np.sqrt(np.mean(x * x, axis=1) + eps)
+    sample = (np.arange(M) // rows_per_sample) if rows_per_sample else np.zeros(M, dtype=np.int64)
+
+    def per_row(v):
+        if v is None:
+            return np.zeros((M, C), dtype=np.float64)
+        return np.asarray(v, dtype=np.float64).reshape(-1, C)[sample]
+
+    u = x * rstd[:, None] * (1.0 + per_row(scale)) + per_row(shift)
+    return u, rstd
+
+
+def adaln_quantize(x, shift=None, scale=None, eps: float = 1e-6, rows_per_sample: int = 0,
+                   g: np.float32 | None = None):
+    """The quantiser with the adaLN prologue: the modulated row is rounded once to bf16 (the value an
+    unfused model would hold in memory) and quantised by the block rule.  With g None the tensor scale
+    is amax(|u|) / 2688 of that bf16 tensor.  Returns ((codes, scales, g), u_bf16, rstd)."""
+    u, rstd = adaln_modulate(x, shift, scale, eps, rows_per_sample)
+    ub = to_bf16_round(u)
+    return quantize(ub, g), ub, rstd
+
+
 def rel_err_normwise(got: np.ndarray, ref: np.ndarray) -> float:
     """max |got - ref| / max |ref| over the whole tensor."""
     ref = np.asarray(ref, dtype=np.float64)

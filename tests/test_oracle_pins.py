@@ -412,3 +412,74 @@ def test_fake_quantize_element_rounding_matches_ml_dtypes():
     e = v.astype(ml_dtypes.float4_e2m1fn).astype(np.float32)
     ref = (e * d).astype(np.float32).astype(ml_dtypes.bfloat16).astype(np.float32)
     np.testing.assert_array_equal(y, ref)
+
+
+# ------------------------------------------------------------------------------------------
+# adaLN prologue (RMSNorm, then (1 + scale) and shift per sample)
+# ------------------------------------------------------------------------------------------
+
+def test_adaln_without_modulation_is_torch_rms_norm():
+    """scale = shift = 0 reduces the prologue to RMSNorm without a weight: torch's own rms_norm in fp64."""
+    import torch
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((7, 96)) * np.array([10.0 ** rng.integers(-3, 3) for _ in range(7)])[:, None]
+    for eps in (1e-6, 0.5):
+        u, rstd = O.adaln_modulate(x, np.zeros(96), np.zeros(96), eps=eps)
+        ref = torch.nn.functional.rms_norm(torch.from_numpy(x), (96,), eps=eps).numpy()
+        np.testing.assert_allclose(u, ref, rtol=1e-13, atol=0)
+        np.testing.assert_allclose(x * rstd[:, None], ref, rtol=1e-13, atol=0)
+
+
+def test_adaln_closed_forms():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((5, 64))
+    shift = rng.standard_normal(64)
+    # scale = -1 removes the normalised row: u is the shift, whatever x is
+    u, _ = O.adaln_modulate(x, shift, -np.ones(64))
+    np.testing.assert_array_equal(u, np.broadcast_to(shift, u.shape))
+    # a constant row c normalises to c / sqrt(c^2 + eps); (1 + 0.5) * that + 0.25 rounds to bf16 1.75
+    c = np.full((2, 32), 2.0)
+    c[1] = -2.0
+    u, rstd = O.adaln_modulate(c, np.full(32, 0.25), np.full(32, 0.5), eps=1e-6)
+    np.testing.assert_allclose(rstd, 1.0 / math.sqrt(4.0 + 1e-6), rtol=1e-15)
+    np.testing.assert_array_equal(O.to_bf16_round(u)[0], 1.75)
+    np.testing.assert_array_equal(O.to_bf16_round(u)[1], -1.25)    # -1.5 + 0.25: the shift is not scaled
+    # mean square of an unmodulated row is ms / (ms + eps)
+    u, _ = O.adaln_modulate(x, None, None, eps=0.3)
+    ms = np.mean(x * x, axis=1)
+    np.testing.assert_allclose(np.mean(u * u, axis=1), ms / (ms + 0.3), rtol=1e-13)
+
+
+def test_adaln_is_invariant_to_row_scale_when_eps_vanishes():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((4, 128))
+    sh, sc = rng.standard_normal(128), rng.standard_normal(128)
+    u1, r1 = O.adaln_modulate(x, sh, sc, eps=1e-30)
+    u2, r2 = O.adaln_modulate(x * 1024.0, sh, sc, eps=1e-30)
+    np.testing.assert_allclose(u1, u2, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(r1, r2 * 1024.0, rtol=1e-12)
+
+
+def test_adaln_sample_of_each_row():
+    """rows [b*L, (b+1)*L) take sample b's vectors; L = 0 gives every row sample 0."""
+    x = np.random.default_rng(6).standard_normal((7, 16))
+    shift = np.arange(1, 4, dtype=np.float64)[:, None] * np.ones((3, 16))
+    u, _ = O.adaln_modulate(x, shift, -np.ones((3, 16)), rows_per_sample=3)
+    np.testing.assert_array_equal(u[:, 0], [1, 1, 1, 2, 2, 2, 3])
+    u, _ = O.adaln_modulate(x, shift, -np.ones((3, 16)), rows_per_sample=0)
+    np.testing.assert_array_equal(u[:, 0], np.ones(7))
+
+
+def test_adaln_quantize_codes_approximate_the_modulated_row():
+    """Each dequantised element is within half a code step of the bf16 modulated value (the block rule's
+    error bound, with the 6-saturation of the E4M3 rounding allowed for), and g follows from amax(u)."""
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((33, 256)).astype(np.float32)
+    sh, sc = 0.5 * rng.standard_normal(256), 0.5 * rng.standard_normal(256)
+    (codes, scales, g), ub, rstd = O.adaln_quantize(x, sh, sc)
+    assert g == np.float32(np.max(np.abs(ub)) / np.float32(2688.0))
+    d = O.e4m3_decode(scales) * np.float64(g)
+    err = np.abs(O.dequantize_exact(codes, scales, g) - ub).reshape(33, 16, 16)
+    amax_b = np.abs(ub).reshape(33, 16, 16).max(axis=2)
+    bound = np.maximum(d, 0) + np.maximum(amax_b - 6 * d, 0)    # one step of 2 * d at most, or the clip
+    assert np.all(err.max(axis=2) <= bound + 1e-12)
