@@ -502,6 +502,15 @@ def op_case(name):
         scale = torch.full((1,), 3.0 / 2688.0, dtype=torch.float32, device=dev)
         return (lambda: B.fake_quantize(x, y=y, scale=scale, static=static)), 4.0 * rows * cols, "GB/s (4 B/elem)"
 
+    def adaln(static=False):
+        case = W.adaln_2k()
+        x, sh, sc = case.x.to(dev), case.shift[0].to(dev), case.scale[0].to(dev)
+        rows, cols = case.x.shape
+        q = B.QTensor.empty(rows, cols)
+        q.g.fill_(3.0 / 2688.0)
+        fn = lambda: B.adaln_quantize(x, sh, sc, eps=case.eps, out=q, static=static)
+        return fn, 2.5625 * rows * cols + 4.0 * cols, "GB/s (2.5625 B/elem)"
+
     def amax(rows, cols):
         x = W.to_bf16(W.normal(np.random.default_rng(0), (rows, cols))).to(dev)
         o = torch.empty(1, dtype=torch.float32, device=dev)
@@ -527,6 +536,8 @@ def op_case(name):
         "fakeq_2k_static": lambda: fakeq(M2, W.HIDDEN, static=True),
         "quant_text_static": lambda: quant(W.HIDDEN, W.TEXT_K, static=True),
         "amax_2k": lambda: amax(M2, W.HIDDEN),
+        "adaln_2k": lambda: adaln(),
+        "adaln_2k_static": lambda: adaln(static=True),
     }
     return table[name]
 

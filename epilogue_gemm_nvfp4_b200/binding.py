@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libnvfp4.so")
 EXPORTS = ("nvfp4_quantize", "nvfp4_linear", "nvfp4_dequantize", "nvfp4_amax", "nvfp4_scale_bytes",
            "nvfp4_scale_offset", "nvfp4_get_device_error", "nvfp4_linear_tile_n", "nvfp4_linear_split_k",
            "nvfp4_status_string", "nvfp4_version", "nvfp4_linear_noalloc", "nvfp4_linear_noalloc_scratch_bytes",
-           "nvfp4_fake_quantize")
+           "nvfp4_fake_quantize", "nvfp4_adaln_quantize")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_MISALIGNED, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_SCRATCH_LIMIT = range(7)
 EPI_BIAS, EPI_QKNORM, EPI_GATED_SILU, EPI_RESID_GATE = range(4)
@@ -38,6 +38,12 @@ class CEpilogue(ctypes.Structure):
                 ("q_col0", ctypes.c_int64), ("k_col0", ctypes.c_int64), ("qk_cols", ctypes.c_int64),
                 ("residual", ctypes.c_void_p), ("ld_residual", ctypes.c_int64), ("gate", ctypes.c_void_p),
                 ("out_nvfp4", ctypes.c_int32), ("out_amax", ctypes.c_void_p)]
+
+
+class CAdaln(ctypes.Structure):
+    _fields_ = [("shift", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("ld_mod", ctypes.c_int64),
+                ("rows_per_sample", ctypes.c_int64), ("eps", ctypes.c_float), ("rstd", ctypes.c_void_p),
+                ("u_out", ctypes.c_void_p), ("ld_u", ctypes.c_int64)]
 
 
 class NvFp4Error(RuntimeError):
@@ -60,6 +66,7 @@ def load() -> ctypes.CDLL:
     P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
     TP = ctypes.POINTER(CTensor)
     EP = ctypes.POINTER(CEpilogue)
+    AP = ctypes.POINTER(CAdaln)
     sig = {
         "nvfp4_quantize": (I32, [P, I64, I64, I64, I32, TP, P]),
         "nvfp4_linear": (I32, [TP, TP, EP, P, I64, TP, P]),
@@ -67,6 +74,7 @@ def load() -> ctypes.CDLL:
         "nvfp4_linear_noalloc_scratch_bytes": (SZ, []),
         "nvfp4_dequantize": (I32, [TP, P, I64, P]),
         "nvfp4_fake_quantize": (I32, [P, I64, I64, I64, I32, P, P, I64, P]),
+        "nvfp4_adaln_quantize": (I32, [P, I64, I64, I64, AP, I32, TP, P]),
         "nvfp4_amax": (I32, [P, I64, I64, I64, P, P]),
         "nvfp4_scale_bytes": (SZ, [I64, I64]),
         "nvfp4_scale_offset": (I64, [I64, I64, I64]),
@@ -176,6 +184,34 @@ def fake_quantize(x: torch.Tensor, y: torch.Tensor | None = None, g: float | tor
     _check(load().nvfp4_fake_quantize(_ptr(x), rows, cols, x.stride(0), int(compute), _ptr(scale), _ptr(y),
                                       y.stride(0), _stream(stream)), "nvfp4_fake_quantize")
     return y, scale
+
+
+def adaln_quantize(x: torch.Tensor, shift: torch.Tensor | None = None, scale: torch.Tensor | None = None,
+                   eps: float = 1e-6, rows_per_sample: int = 0, out: QTensor | None = None,
+                   g: float | torch.Tensor | None = None, static: bool = False, rstd: torch.Tensor | None = None,
+                   u_out: torch.Tensor | None = None, stream=None) -> QTensor:
+    """NVFP4 of u = bf16(RMSNorm(x) * (1 + scale) + shift) through nvfp4_adaln_quantize.  shift / scale are
+    bf16 [cols] or [samples, cols] (row r uses sample r // rows_per_sample).  The tensor scale follows
+    ``quantize``: computed on the device by default, ``g`` given, or ``static`` (out.g as it is).
+    ``rstd`` (fp32 [rows]) and ``u_out`` (bf16 [rows, cols]) receive the per-row 1/rms and u when given."""
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    out = QTensor.empty(rows, cols, x.device) if out is None else out
+    if g is not None:
+        out.g.copy_(torch.as_tensor(g, dtype=torch.float32).reshape(1))
+    compute = g is None and not static
+    mods = [m for m in (shift, scale) if m is not None]
+    for m in mods:
+        assert m.is_cuda and m.dtype == torch.bfloat16 and m.stride(-1) == 1
+    ld_mod = mods[0].stride(0) if mods and mods[0].dim() == 2 else cols
+    if len(mods) == 2 and mods[0].dim() == 2:
+        assert mods[1].dim() == 2 and mods[1].stride(0) == ld_mod, "shift and scale need the same sample stride"
+    desc = CAdaln(_ptr(shift), _ptr(scale), int(ld_mod), int(rows_per_sample), float(eps), _ptr(rstd),
+                  _ptr(u_out), u_out.stride(0) if u_out is not None else 0)
+    ct = out.c()
+    _check(load().nvfp4_adaln_quantize(_ptr(x), rows, cols, x.stride(0), ctypes.byref(desc), int(compute),
+                                       ctypes.byref(ct), _stream(stream)), "nvfp4_adaln_quantize")
+    return out
 
 
 def dequantize(q: QTensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:

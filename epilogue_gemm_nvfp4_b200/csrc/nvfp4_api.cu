@@ -10,6 +10,7 @@
 #include <utility>
 
 #include "nvfp4.h"
+#include "adaln.cuh"
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
 #include "ptx.cuh"
@@ -416,6 +417,57 @@ nvfp4_status nvfp4_fake_quantize(const void* x, int64_t rows, int64_t cols, int6
     const int grid = resident_grid(fk, 256, tasks, 8, st->sm_count);
     fk<<<grid, 256, 0, s>>>(xb, rows, cols, ldx, tensor_scale, static_cast<__nv_bfloat16*>(y), ldy);
   }
+  return launch_status();
+}
+
+nvfp4_status nvfp4_adaln_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, const nvfp4_adaln_desc* ada,
+                                  int32_t compute_scale, const nvfp4_tensor* out, nvfp4_stream_t stream) {
+  if (!x || !ada || !out || rows < 0 || cols <= 0 || ldx < cols) return NVFP4_ERR_INVALID_ARG;
+  if (!(ada->eps > 0.0f) || ada->eps > 3.0e38f || ada->rows_per_sample < 0) return NVFP4_ERR_INVALID_ARG;
+  const bool per_sample = ada->rows_per_sample > 0 && ada->rows_per_sample < rows;
+  if (per_sample && (ada->shift || ada->scale) && ada->ld_mod < cols) return NVFP4_ERR_INVALID_ARG;
+  if (ada->u_out && ada->ld_u < cols) return NVFP4_ERR_INVALID_ARG;
+  if (nvfp4_status e = check_tensor(out, true, 8)) return e;
+  if (out->rows != rows || out->cols != cols) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(x) || (ldx * 2) % 16) return NVFP4_ERR_MISALIGNED;
+  if ((ada->shift && !aligned16(ada->shift)) || (ada->scale && !aligned16(ada->scale)) ||
+      (per_sample && (ada->ld_mod * 2) % 16) || (ada->rstd && !aligned4(ada->rstd)) ||
+      (ada->u_out && (!aligned16(ada->u_out) || (ada->ld_u * 2) % 16)))
+    return NVFP4_ERR_MISALIGNED;
+  DeviceState* st;
+  if (nvfp4_status e = device_state(&st)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  AdalnArgs a{};
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.rows = rows;
+  a.cols = cols;
+  a.ldx = ldx;
+  a.shift = static_cast<const __nv_bfloat16*>(ada->shift);
+  a.scale = static_cast<const __nv_bfloat16*>(ada->scale);
+  a.ld_mod = ada->ld_mod;
+  a.rows_per_sample = per_sample ? ada->rows_per_sample : 0;
+  a.eps = ada->eps;
+  a.g_src = out->tensor_scale;
+  a.codes = static_cast<uint8_t*>(out->codes);
+  a.ld_codes = ld_codes_of(out);
+  a.scales = static_cast<uint8_t*>(out->scales);
+  a.k_atoms = k_atoms_of(cols);
+  a.rstd = ada->rstd;
+  a.u = static_cast<__nv_bfloat16*>(ada->u_out);
+  a.ld_u = ada->ld_u;
+  a.tensor_scale = out->tensor_scale;
+  const bool vec32 = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx * 2) % 32 == 0;
+  // dynamic scale: the amax pass walks the rows front to back, the quantise pass back to front
+  auto qk = compute_scale ? (vec32 ? adaln_quantize_kernel<false, true, true> : adaln_quantize_kernel<false, true, false>)
+                          : (vec32 ? adaln_quantize_kernel<false, false, true> : adaln_quantize_kernel<false, false, false>);
+  if (compute_scale) {
+    if (nvfp4_status e = amax_state_for(s, &a.state)) return e;
+    auto ak = vec32 ? adaln_quantize_kernel<true, false, true> : adaln_quantize_kernel<true, false, false>;
+    const int agrid = resident_grid(ak, 256, rows, 8, st->sm_count);
+    ak<<<agrid, 256, 0, s>>>(a);
+  }
+  const int qgrid = resident_grid(qk, 256, rows + 1, 8, st->sm_count);
+  qk<<<qgrid, 256, 0, s>>>(a);
   return launch_status();
 }
 

@@ -32,6 +32,18 @@ __device__ __forceinline__ uint32_t bf16x2_absmax_bits(uint32_t w) {
 // so the reduction runs on integers and one atomicMax per CTA publishes the fp32 bit pattern.
 // ------------------------------------------------------------------------------------------
 
+// max of one value per thread over the CTA (valid in thread 0); blockDim.x <= 1024
+__device__ __forceinline__ uint32_t cta_max_u32(uint32_t m) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __shared__ uint32_t red[32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) m = max(m, red[w]);
+  return m;
+}
+
 // max over this CTA's share of the matrix of the bf16 magnitude bits (valid in thread 0)
 __device__ __forceinline__ uint32_t block_absmax_bits(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols,
                                                       int64_t ldx) {
@@ -67,20 +79,28 @@ __device__ __forceinline__ uint32_t block_absmax_bits(const __nv_bfloat16* __res
       }
     }
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  __shared__ uint32_t red[8];
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-  __syncthreads();
-  if (threadIdx.x == 0)
-    for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) m = max(m, red[w]);
-  return m;
+  return cta_max_u32(m);
 }
 
 __global__ void __launch_bounds__(256) amax_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
                                                    int64_t cols, int64_t ldx, unsigned int* __restrict__ out_bits) {
   const uint32_t m = block_absmax_bits(x, rows, cols, ldx);
   if (threadIdx.x == 0 && m) atomicMax(out_bits, m << 16);  // bf16 magnitude -> fp32 bit pattern
+}
+
+// Thread 0 of every CTA of a grid: publish the CTA's max (bf16 magnitude bits), then take a ticket;
+// the CTA with the last ticket writes g = amax / 2688 (1 for an all-zero tensor) and puts the
+// per-stream state {amax bits, CTAs done} back to zero for the next call on the stream.
+__device__ __forceinline__ void finish_tensor_scale(uint32_t m, unsigned int* state, float* tensor_scale) {
+  if (m) atomicMax(&state[0], m << 16);  // bf16 magnitude -> fp32 bit pattern
+  __threadfence();
+  if (atomicAdd(&state[1], 1u) == gridDim.x - 1) {
+    __threadfence();
+    const float amax = __uint_as_float(atomicOr(&state[0], 0u));
+    *tensor_scale = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, kTensorScaleDivisor);
+    state[0] = 0u;
+    state[1] = 0u;
+  }
 }
 
 // The same reduction, finished in place: the last CTA to finish writes the tensor decode scale
@@ -92,17 +112,7 @@ __global__ void __launch_bounds__(256) amax_scale_kernel(const __nv_bfloat16* __
                                                          int64_t cols, int64_t ldx, unsigned int* __restrict__ state,
                                                          float* __restrict__ tensor_scale) {
   const uint32_t m = block_absmax_bits(x, rows, cols, ldx);
-  if (threadIdx.x == 0) {
-    if (m) atomicMax(&state[0], m << 16);
-    __threadfence();
-    if (atomicAdd(&state[1], 1u) == gridDim.x - 1) {
-      __threadfence();
-      const float amax = __uint_as_float(atomicOr(&state[0], 0u));
-      *tensor_scale = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, kTensorScaleDivisor);
-      state[0] = 0u;
-      state[1] = 0u;
-    }
-  }
+  if (threadIdx.x == 0) finish_tensor_scale(m, state, tensor_scale);
 }
 
 // The block rule for one 16-element block, given its amax and the tensor decode scale g:
@@ -114,6 +124,47 @@ __device__ __forceinline__ uint32_t block_scale(float amax_b, float g, float& in
   const float d = __fmul_rn(e4m3_to_float(s), g);
   inv = (d == 0.0f) ? 0.0f : __frcp_rn(d);
   return s;
+}
+
+// The block rule on one 16-element block held as 8 bf16x2 words (element 2i in the low half of word
+// i): returns the E4M3 scale byte and writes the 16 codes two per byte, element 2i in the low nibble
+// (all codes 0 when d == 0).  `inv` is 1/d, 0 when d == 0.
+__device__ __forceinline__ uint32_t quantize_block16(const uint32_t (&w)[8], float g, uint32_t (&packed)[2],
+                                                     float& inv) {
+  uint32_t m2 = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m2 = __vmaxu2(m2, w[i] & 0x7FFF7FFFu);
+  const uint32_t mb = max(m2 & 0xFFFFu, m2 >> 16);
+  const uint32_t sc = block_scale(__uint_as_float(mb << 16), g, inv);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float q[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      q[2 * i] = __fmul_rn(__uint_as_float(w[4 * h + i] << 16), inv);
+      q[2 * i + 1] = __fmul_rn(__uint_as_float(w[4 * h + i] & 0xFFFF0000u), inv);
+    }
+    packed[h] = (inv == 0.0f) ? 0u : e2m1x8(q);
+  }
+  return sc;
+}
+
+// Quantise one block per lane and store it: lane `lane` of the warp holds block `blk` of a row whose
+// codes start at `crow` and whose scales start at `srow` (the row's first scale word in the atom
+// layout).  Every lane of the warp takes part (the scale bytes of four lanes form one 32-bit word);
+// lanes with valid == false store nothing.
+__device__ __forceinline__ void store_block16(const uint32_t (&w)[8], float g, int blk, bool valid, int lane,
+                                              uint8_t* crow, uint8_t* srow) {
+  uint32_t packed[2];
+  float inv;
+  uint32_t sc = quantize_block16(w, g, packed, inv);
+  if (!valid) sc = 0;
+  if (valid) *reinterpret_cast<uint2*>(crow + static_cast<int64_t>(blk) * 8) = make_uint2(packed[0], packed[1]);
+  const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
+  const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
+  const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
+  if ((lane & 3) == 0 && valid)
+    *reinterpret_cast<uint32_t*>(srow + static_cast<int64_t>(blk >> 2) * 512) = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -177,32 +228,7 @@ __global__ void __launch_bounds__(256, 6) quantize_kernel(const __nv_bfloat16* _
       for (int u = 0; u < kQuantUnroll; ++u) {
         if (st + u >= st_end) break;  // warp-uniform
         const int blk = (st + u) * 32 + lane;
-        const bool valid = blk < bpr;
-        uint32_t m2 = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m2 = __vmaxu2(m2, w[u][i] & 0x7FFF7FFFu);
-        const uint32_t mb = max(m2 & 0xFFFFu, m2 >> 16);
-        float inv;
-        uint32_t sc = block_scale(__uint_as_float(mb << 16), g, inv);
-        uint32_t packed[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float q[8];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            q[2 * i] = __fmul_rn(__uint_as_float(w[u][4 * h + i] << 16), inv);
-            q[2 * i + 1] = __fmul_rn(__uint_as_float(w[u][4 * h + i] & 0xFFFF0000u), inv);
-          }
-          packed[h] = (inv == 0.0f) ? 0u : e2m1x8(q);
-        }
-        if (!valid) sc = 0;
-        if (valid) *reinterpret_cast<uint2*>(crow + static_cast<int64_t>(blk) * 8) = make_uint2(packed[0], packed[1]);
-        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
-        const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
-        const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
-        if ((lane & 3) == 0 && valid)
-          *reinterpret_cast<uint32_t*>(srow + static_cast<int64_t>(blk >> 2) * 512) =
-              sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        store_block16(w[u], g, blk, blk < bpr, lane, crow, srow);
       }
     }
   }
@@ -265,26 +291,16 @@ __global__ void __launch_bounds__(256, 6) fake_quantize_kernel(const __nv_bfloat
         if (st + u >= st_end) break;  // warp-uniform
         const int blk = (st + u) * 32 + lane;
         if (blk >= bpr) continue;
-        uint32_t m2 = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m2 = __vmaxu2(m2, w[u][i] & 0x7FFF7FFFu);
-        const uint32_t mb = max(m2 & 0xFFFFu, m2 >> 16);
+        uint32_t packed[2];
         float inv;
-        const uint32_t sc = block_scale(__uint_as_float(mb << 16), g, inv);
+        const uint32_t sc = quantize_block16(w[u], g, packed, inv);
         const float d = __fmul_rn(e4m3_to_float(sc), g);
         uint32_t o[8];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          float q[8];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            q[2 * i] = __fmul_rn(__uint_as_float(w[u][4 * h + i] << 16), inv);
-            q[2 * i + 1] = __fmul_rn(__uint_as_float(w[u][4 * h + i] & 0xFFFF0000u), inv);
-          }
-          const uint32_t codes8 = (inv == 0.0f) ? 0u : e2m1x8(q);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t byte = (codes8 >> (8 * i)) & 0xFFu;
+            const uint32_t byte = (packed[h] >> (8 * i)) & 0xFFu;
             const __nv_bfloat16 lo = __float2bfloat16_rn(__fmul_rn(e2m1_to_float(byte & 0xFu), d));
             const __nv_bfloat16 hi = __float2bfloat16_rn(__fmul_rn(e2m1_to_float(byte >> 4), d));
             o[4 * h + i] = static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |

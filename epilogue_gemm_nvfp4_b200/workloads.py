@@ -152,6 +152,30 @@ def case_text(T, K=TEXT_K, N=HIDDEN, seed=0, w_std=0.005, b_std=0.01, zero_rows=
     return LinearCase(name, to_bf16(x), to_bf16(w), to_bf16(b), "bias")
 
 
+@dataclass
+class AdalnCase:
+    """A DiT hidden state x [M, C] and its adaLN vectors shift, scale [S, C] (one pair per sample;
+    row r belongs to sample r // rows_per_sample, or to sample 0 when rows_per_sample is 0)."""
+    name: str
+    x: torch.Tensor
+    shift: torch.Tensor
+    scale: torch.Tensor
+    rows_per_sample: int = 0
+    eps: float = 1e-6
+
+
+def case_adaln(M, C=HIDDEN, samples=1, seed=0, outlier_frac=0.01, outlier_factor=30.0, mod_std=0.5,
+               name="adaln") -> AdalnCase:
+    """x N(0,1) with 1% outlier channels x30 (as the QKV input); shift, scale N(0, mod_std^2) per sample."""
+    rng = np.random.default_rng(seed)
+    x = normal(rng, (M, C))
+    x = with_outlier_columns(rng, x, int(round(outlier_frac * C)), outlier_factor)
+    shift = normal(rng, (samples, C), mod_std)
+    scale = normal(rng, (samples, C), mod_std)
+    L = 0 if samples == 1 else -(-M // samples)
+    return AdalnCase(name, to_bf16(x), to_bf16(shift), to_bf16(scale), L)
+
+
 # ---- the named workloads -------------------------------------------------------------------
 
 def tiny(seed=0) -> LinearCase:
@@ -182,6 +206,11 @@ def block_2k(seed=7, M=IMG_TOKENS_2K + PROMPT_T) -> dict:
         up=case_ffn_up(M, seed=seed + 2, name="block2k_up"),
         down=case_ffn_down(M, seed=seed + 3, with_x=False, name="block2k_down"),
     )
+
+
+def adaln_2k(seed=7, M=IMG_TOKENS_2K + PROMPT_T) -> AdalnCase:
+    """The hidden state in front of the QKV / FFN-up products at 2048^2, with its adaLN modulation."""
+    return case_adaln(M, seed=seed, name="adaln_2048sq")
 
 
 def flops(case: LinearCase) -> float:

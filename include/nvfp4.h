@@ -199,6 +199,54 @@ NVFP4_API nvfp4_status nvfp4_fake_quantize(const void* x, int64_t rows, int64_t 
                                            int32_t compute_scale, float* tensor_scale, void* y, int64_t ldy,
                                            nvfp4_stream_t stream);
 
+/*
+ * The adaLN prologue of a DiT block, fused into the quantiser.  RMSNorm is one of the small ops that
+ * follow the big products ("Serving sub-second Ideogram v4 without quality loss", paragraph on kernel
+ * fusion); adaLN modulates the hidden state with vectors generated at run time ("Quantizing a
+ * Dual-Branch Flow-Matching Diffusion Transformer for Consumer GPUs", related-work paragraph on W8A8).
+ * For row r of x and its sample b = r / rows_per_sample:
+ *   rstd[r] = 1 / sqrt(mean_k x[r,k]^2 + eps)
+ *   u[r,k]  = bf16( x[r,k] * rstd[r] * (1 + scale[b,k]) + shift[b,k] )
+ * and u is quantised by the rule of nvfp4_quantize, so the codes equal nvfp4_quantize(u) bit for bit.
+ *   shift, scale:     bf16 vectors of `cols` elements per sample, sample b at element offset b * ld_mod,
+ *                     ceil(rows / rows_per_sample) samples (one when rows_per_sample is 0);
+ *                     NULL = no shift / multiplier 1.
+ *   ld_mod:           elements between samples (>= cols; read only when rows_per_sample > 0).
+ *   rows_per_sample:  rows [b * L, (b + 1) * L) use sample b; 0 (or >= rows) = sample 0 for every row.
+ *   eps:              > 0.
+ *   rstd:             device fp32 [rows] or NULL: receives rstd[r].
+ *   u_out, ld_u:      bf16 [rows, ld_u] or NULL: receives u (the values that were quantised).
+ * Arithmetic: the sum of squares is an fp32 sum in a fixed order (it does not depend on `rows`); then
+ * rstd = 1 / sqrt(sum / cols + eps), x * rstd and 1 + scale each rounded to fp32, one fused
+ * multiply-add with shift, and one rounding to bf16.
+ */
+typedef struct {
+  const void* shift;
+  const void* scale;
+  int64_t ld_mod;
+  int64_t rows_per_sample;
+  float eps;
+  float* rstd;
+  void* u_out;
+  int64_t ld_u;
+} nvfp4_adaln_desc;
+
+/*
+ * Quantise adaLN(x) (see nvfp4_adaln_desc) to NVFP4 into `out` (out->rows == rows, out->cols == cols).
+ *   compute_scale = 1: g = amax(|u|) / 2688 (1 for an all-zero or empty u) is computed on the device
+ *                      and stored in *out->tensor_scale: two stream-ordered launches of one kernel, an
+ *                      amax pass that computes u and reduces its max (its last CTA writes g), then the
+ *                      quantise pass.  The per-stream state and the rule on graph capture are those of
+ *                      nvfp4_quantize.
+ *   compute_scale = 0: the g already stored in *out->tensor_scale is used; one launch.
+ * Rules: cols % 16 == 0; x, ldx*2, shift, scale, ld_mod*2 (when read), u_out, ld_u*2, codes and scales
+ * 16-byte aligned; rstd 4-byte aligned; ld_codes a multiple of 8.  Rows of up to 4608 elements are read
+ * from memory once (twice with compute_scale = 1); longer rows once more per pass.
+ */
+NVFP4_API nvfp4_status nvfp4_adaln_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx,
+                                            const nvfp4_adaln_desc* ada, int32_t compute_scale,
+                                            const nvfp4_tensor* out, nvfp4_stream_t stream);
+
 /* Dequantise t to bf16 [t->rows, ld_out]: value = e2m1(code) * (e4m3(scale) * g), each product in fp32
  * rounded to nearest even, then rounded to bf16.  Rules as for nvfp4_quantize. */
 NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor* t, void* out_bf16, int64_t ld_out, nvfp4_stream_t stream);

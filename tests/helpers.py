@@ -67,3 +67,18 @@ def assert_requant_close(q, ref, M, K, max_frac=1e-3):
     dc = np.abs(mag(got_c) - mag(rc.astype(np.int64)))
     dc = np.where(same_scale, dc, 0)
     assert dc.max(initial=0) <= 1 and np.mean(dc > 0) <= max_frac, (dc.max(initial=0), np.mean(dc > 0))
+
+
+def assert_quant_arrays_close(got, ref, max_frac=1e-3):
+    """Row-major (codes [M,K] one per byte, scales [M,K/16], g) against the oracle's, when the two inputs
+    may differ in the last bf16 bit: g equal, and every differing scale byte or code one step apart,
+    each kind of difference in at most ``max_frac`` of the entries."""
+    gc, gs, gg = got
+    rc, rs, rg = ref
+    assert gg == rg, (gg, rg)
+    ds = np.abs(gs.astype(np.int64) - rs.astype(np.int64))
+    assert ds.max(initial=0) <= 1 and np.mean(ds > 0) <= max_frac, (ds.max(initial=0), np.mean(ds > 0))
+    mag = lambda c: np.where(c & 8, -(c & 7), c & 7)
+    dc = np.abs(mag(gc.astype(np.int64)) - mag(rc.astype(np.int64)))
+    dc = np.where(np.repeat(ds == 0, 16, axis=1), dc, 0)
+    assert dc.max(initial=0) <= 1 and np.mean(dc > 0) <= max_frac, (dc.max(initial=0), np.mean(dc > 0))

@@ -102,6 +102,29 @@ def test_argument_checks_return_before_any_launch(lib):
     assert fq(y=0x10008) == B.ERR_MISALIGNED
     assert fq(ldx=516) == B.ERR_MISALIGNED
     assert fq(g=0x10001) == B.ERR_MISALIGNED
+    # adaLN prologue of the quantiser
+    ok = dict(shift=0x10000, scale=0x10000, ld_mod=512, rows_per_sample=0, eps=1e-6, rstd=0x10000,
+              u_out=0x10000, ld_u=512)
+
+    def ada(x=0x10000, rows=4, cols=512, ldx=512, t=t, **kw):
+        d = B.CAdaln(**dict(ok, **kw))
+        return lib.nvfp4_adaln_quantize(x, rows, cols, ldx, ctypes.byref(d), 1, ctypes.byref(t), None)
+    assert lib.nvfp4_adaln_quantize(0x10000, 4, 512, 512, None, 1, ctypes.byref(t), None) == B.ERR_INVALID_ARG
+    assert ada(x=None) == B.ERR_INVALID_ARG
+    assert ada(eps=0.0) == B.ERR_INVALID_ARG
+    assert ada(eps=float("nan")) == B.ERR_INVALID_ARG
+    assert ada(rows_per_sample=-1) == B.ERR_INVALID_ARG
+    assert ada(rows_per_sample=2, ld_mod=256) == B.ERR_INVALID_ARG                        # samples overlap
+    assert ada(ld_u=256) == B.ERR_INVALID_ARG
+    assert ada(rows=5) == B.ERR_INVALID_ARG                                                # out is [4, 512]
+    assert ada(cols=520, ldx=520, ld_u=520, t=_tensor(4, 520)) == B.ERR_UNSUPPORTED_SHAPE
+    assert ada(ldx=516) == B.ERR_MISALIGNED
+    assert ada(shift=0x10008) == B.ERR_MISALIGNED
+    assert ada(scale=0x10004) == B.ERR_MISALIGNED
+    assert ada(rows_per_sample=2, ld_mod=516) == B.ERR_MISALIGNED
+    assert ada(rstd=0x10002) == B.ERR_MISALIGNED
+    assert ada(u_out=0x10008) == B.ERR_MISALIGNED
+    assert ada(ld_u=516) == B.ERR_MISALIGNED
 
 
 @pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-device path")
@@ -118,7 +141,7 @@ def test_ctypes_structs_match_the_header(tmp_path):
     import subprocess
     if shutil.which("gcc") is None:
         pytest.skip("gcc not available")
-    structs = {"nvfp4_tensor": B.CTensor, "nvfp4_epilogue_desc": B.CEpilogue}
+    structs = {"nvfp4_tensor": B.CTensor, "nvfp4_epilogue_desc": B.CEpilogue, "nvfp4_adaln_desc": B.CAdaln}
     lines = ['#include <stdio.h>', '#include "nvfp4.h"', "int main(void) {"]
     for cname, py in structs.items():
         lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
