@@ -140,14 +140,19 @@ def test_adaln_rows_do_not_depend_on_their_neighbours(lib):
 
 
 def test_adaln_quantize_empty_rows(lib):
-    # zero-row views of real buffers, so that every pointer is valid
-    x = torch.empty((1, 512), dtype=torch.bfloat16, device="cuda")[:0]
-    q = B.QTensor(torch.empty((1, 256), dtype=torch.uint8, device="cuda")[:0],
-                  torch.empty(512, dtype=torch.uint8, device="cuda"),
-                  torch.zeros(1, dtype=torch.float32, device="cuda"), 0, 512)
-    B.adaln_quantize(x, out=q)
+    """rows == 0: nothing is encoded and the dynamic scale is 1.  Called through the C ABI with real
+    buffers (torch reports a null data pointer for a tensor with no elements)."""
+    import ctypes
+    x = torch.empty((1, 512), dtype=torch.bfloat16, device="cuda")
+    codes = torch.empty((1, 256), dtype=torch.uint8, device="cuda")
+    scales = torch.empty(512, dtype=torch.uint8, device="cuda")
+    g = torch.zeros(1, dtype=torch.float32, device="cuda")
+    t = B.CTensor(codes.data_ptr(), scales.data_ptr(), g.data_ptr(), 0, 512, 256)
+    d = B.CAdaln(None, None, 512, 0, 1e-6, None, None, 0)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert lib.nvfp4_adaln_quantize(x.data_ptr(), 0, 512, 512, ctypes.byref(d), 1, ctypes.byref(t), stream) == B.OK
     torch.cuda.synchronize()
-    assert q.g.item() == 1.0
+    assert g.item() == 1.0
 
 
 def test_adaln_full_size_sampled_rows(lib):
