@@ -367,6 +367,51 @@ def adaln_quantize(x, shift=None, scale=None, eps: float = 1e-6, rows_per_sample
     return quantize(ub, g), ub, rstd
 
 
+# ---------------------------------------------------------------------------------------------
+# W8A8 INT8 linear (the other format the pages compare against NVFP4)
+# ---------------------------------------------------------------------------------------------
+
+def smoothquant_factors(act_absmax, w, alpha: float = 0.5):
+    """SmoothQuant migration strength alpha ("Quantizing a Dual-Branch Flow-Matching Diffusion Transformer
+    for Consumer GPUs", section on the method: the smoothing vector lambda_j = s_j^alpha /
+    max_i |W_ij|^(1 - alpha) divides the activations' input channel j and multiplies the weights').
+    act_absmax: per-input-channel max |x| from calibration [K]; w: [N, K].  A channel whose activation
+    or weight column is all zero keeps lambda = 1.  Returned as fp32 (the value the kernels receive)."""
+    s = np.asarray(act_absmax, dtype=np.float64)
+    wmax = np.max(np.abs(np.asarray(w, dtype=np.float64)), axis=0)
+    ok = (s > 0) & (wmax > 0)
+    lam = np.ones_like(s)
+    lam[ok] = s[ok] ** alpha / wmax[ok] ** (1.0 - alpha)
+    return lam.astype(F32)
+
+
+def int8_quantize_rows(x, smooth=None):
+    """Symmetric per-row INT8 ([Dual-Branch], method: per-token dynamic activations and per-output-row
+    weights).  Each step is one binary32 operation rounded to nearest even:
+        x'  = x / smooth[k]         (when a smoothing vector is given)
+        s   = max_k |x'| / 127      (1 for an all-zero row)
+        q   = clamp(RNE(x' / s), -127, 127)
+    x float32 [M, K] -> (q int8 [M, K], s float32 [M])."""
+    x = np.asarray(x, dtype=F32)
+    if smooth is not None:
+        x = (x / np.asarray(smooth, dtype=F32)[None, :]).astype(F32)
+    amax = np.max(np.abs(x), axis=1).astype(F32) if x.shape[1] else np.zeros(x.shape[0], F32)
+    s = np.where(amax == 0, F32(1.0), (amax / F32(127.0)).astype(F32)).astype(F32)
+    v = (x / s[:, None]).astype(F32)
+    q = np.clip(np.rint(v), -127, 127).astype(np.int8)      # rint: ties to even
+    return q, s
+
+
+def int8_linear(qa, sa, qw, sw, bias=None):
+    """y[m,n] = (sum_k qa[m,k] * qw[n,k]) * sa[m] * sw[n] + bias[n]: the integer product exactly (int64),
+    the scaling in fp64.  Returns (y fp64, y rounded to bf16)."""
+    acc = np.asarray(qa, dtype=np.int64) @ np.asarray(qw, dtype=np.int64).T
+    y = acc.astype(np.float64) * np.asarray(sa, np.float64)[:, None] * np.asarray(sw, np.float64)[None, :]
+    if bias is not None:
+        y = y + np.asarray(bias, dtype=np.float64)[None, :]
+    return y, to_bf16_round(y)
+
+
 def rel_err_normwise(got: np.ndarray, ref: np.ndarray) -> float:
     """max |got - ref| / max |ref| over the whole tensor."""
     ref = np.asarray(ref, dtype=np.float64)

@@ -483,3 +483,95 @@ def test_adaln_quantize_codes_approximate_the_modulated_row():
     amax_b = np.abs(ub).reshape(33, 16, 16).max(axis=2)
     bound = np.maximum(d, 0) + np.maximum(amax_b - 6 * d, 0)    # one step of 2 * d at most, or the clip
     assert np.all(err.max(axis=2) <= bound + 1e-12)
+
+
+# ------------------------------------------------------------------------------------------
+# W8A8 INT8 linear
+# ------------------------------------------------------------------------------------------
+
+def test_int8_rows_ties_extremes_and_zero_rows():
+    # amax 127 gives s = 1 exactly, so the codes are x rounded half to even
+    x = np.array([[127.0, 0.5, 1.5, 2.5, -2.5, -0.5, 126.5, -3.49],
+                  [0.0] * 8,
+                  [-4.0, 1.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0]], dtype=np.float32)
+    q, s = O.int8_quantize_rows(x)
+    assert s[0] == 1.0 and s[1] == 1.0
+    assert q[0].tolist() == [127, 0, 2, 2, -2, 0, 126, -3]
+    assert q[1].tolist() == [0] * 8
+    assert q[2, 0] == -127 and s[2] == np.float32(4.0) / np.float32(127.0)
+    assert q[2, 1] == 32                                         # 1 / (4/127) = 31.75 -> 32
+
+
+def test_int8_rows_within_half_a_step_of_the_exact_quotient():
+    """Brute force in exact rationals: every code is a nearest integer to x / s for the fp32 s."""
+    rng = np.random.default_rng(9)
+    x = (rng.standard_t(3, size=(6, 40)) * 10.0 ** rng.integers(-3, 3, size=(6, 1))).astype(np.float32)
+    q, s = O.int8_quantize_rows(x)
+    for r in range(6):
+        amax = max(abs(Fraction(float(v))) for v in x[r])
+        assert abs(Fraction(float(s[r])) - amax / 127) <= Fraction(float(s[r])) * Fraction(1, 2 ** 23)
+        for v, c in zip(x[r], q[r]):
+            e = abs(Fraction(float(v)) / Fraction(float(s[r])) - int(c))
+            assert e <= Fraction(1, 2) + Fraction(1, 2 ** 16), (v, c)
+        assert np.max(np.abs(q[r])) == 127
+
+
+def test_int8_smoothing_divides_each_input_channel():
+    rng = np.random.default_rng(10)
+    x = rng.standard_normal((4, 32)).astype(np.float32)
+    lam = np.ones(32, np.float32)
+    lam[5] = 4.0
+    q1, s1 = O.int8_quantize_rows(x, lam)
+    x2 = x.copy()
+    x2[:, 5] /= 4.0
+    q2, s2 = O.int8_quantize_rows(x2)
+    assert np.array_equal(q1, q2) and np.array_equal(s1, s2)
+
+
+def test_smoothquant_factors_balance_the_channel_ranges():
+    rng = np.random.default_rng(11)
+    w = rng.standard_normal((48, 32)) * 0.02
+    act = np.abs(rng.standard_normal(32)) * 10 + 0.1
+    act[3], w[:, 7] = 0.0, 0.0                                  # dead channels keep lambda = 1
+    lam = O.smoothquant_factors(act, w, 0.5).astype(np.float64)
+    wmax = np.max(np.abs(w), axis=0)
+    live = (act > 0) & (wmax > 0)
+    # alpha = 1/2 gives the activation and weight columns the same range after the migration
+    np.testing.assert_allclose((act / lam)[live], (wmax * lam)[live], rtol=2e-7)
+    assert lam[3] == 1.0 and lam[7] == 1.0
+    # alpha = 1 moves all of it into the weights, alpha = 0 none of the activations' range
+    np.testing.assert_allclose(O.smoothquant_factors(act, w, 1.0)[live], act[live], rtol=1e-7)
+    np.testing.assert_allclose(O.smoothquant_factors(act, w, 0.0)[live], 1.0 / wmax[live], rtol=1e-7)
+    # and the unquantised product is unchanged: (x / lambda) (W lambda)^T = x W^T
+    x = rng.standard_normal((5, 32))
+    np.testing.assert_allclose((x / lam) @ (w * lam).T, x @ w.T, rtol=1e-12, atol=1e-15)
+
+
+def test_int8_linear_exact_integer_product_and_scaling():
+    rng = np.random.default_rng(12)
+    qa = rng.integers(-127, 128, size=(3, 20)).astype(np.int8)
+    qw = rng.integers(-127, 128, size=(4, 20)).astype(np.int8)
+    sa = np.array([0.5, 0.01, 3.0], np.float32)
+    sw = np.array([0.25, 1e-3, 2.0, 7.0], np.float32)
+    bias = np.array([1.0, -1.0, 0.0, 0.5])
+    y, yb = O.int8_linear(qa, sa, qw, sw, bias)
+    for m in range(3):
+        for n in range(4):
+            acc = sum(int(qa[m, k]) * int(qw[n, k]) for k in range(20))
+            want = Fraction(acc) * Fraction(float(sa[m])) * Fraction(float(sw[n])) + Fraction(bias[n])
+            assert abs(Fraction(y[m, n]) - want) <= abs(want) * Fraction(1, 2 ** 50) + Fraction(1, 2 ** 60)
+    np.testing.assert_array_equal(yb, O.to_bf16_round(y))
+
+
+def test_w8a8_error_bound():
+    """|y - x W^T| <= sum_k (|x| e_w + |w| e_x + e_x e_w), e = half a quantisation step per row."""
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((6, 64)).astype(np.float32)
+    w = (rng.standard_normal((8, 64)) * 0.05).astype(np.float32)
+    qa, sa = O.int8_quantize_rows(x)
+    qw, sw = O.int8_quantize_rows(w)
+    y, _ = O.int8_linear(qa, sa, qw, sw)
+    ex, ew = sa.astype(np.float64)[:, None] / 2, sw.astype(np.float64)[:, None] / 2
+    bound = (np.abs(x).astype(np.float64) @ np.ones((64, 8))) * ew.T + ex * (np.ones((6, 64)) @ np.abs(w).T) \
+        + 64 * ex * ew.T
+    assert np.all(np.abs(y - x.astype(np.float64) @ w.astype(np.float64).T) <= bound * (1 + 1e-6))
