@@ -17,6 +17,7 @@ path has no exchange step); the time is the max over ranks and the value counts 
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import os
 import statistics
@@ -43,16 +44,17 @@ BF16_TO_FP4 = 4.0             # nominal dense FP4 / dense bf16 tensor-core rate 
 TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "nvfp4_gemm_up_dram_2048sq.md")
 
 
+#: the sources the up-projection GEMM is built from: its device code and the host code that launches it
+GEMM_SOURCES = ("ptx.cuh", "quantize.cuh", "gemm.cuh", "gemm_pair.cuh", "nvfp4_api.cu")
+
+
 def library_sources_sha256():
-    """sha256 over the library's CUDA sources and header (file name, then bytes, in sorted path order)."""
-    import glob
+    """sha256 over the up GEMM's sources (GEMM_SOURCES: file name, then bytes, in that order)."""
     import hashlib
-    files = sorted(glob.glob(os.path.join(ROOT, "epilogue_gemm_nvfp4_b200", "csrc", "*.cu*")))
-    files.append(os.path.join(ROOT, "include", "nvfp4.h"))
     h = hashlib.sha256()
-    for f in files:
-        h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
+    for name in GEMM_SOURCES:
+        h.update(name.encode())
+        with open(os.path.join(ROOT, "epilogue_gemm_nvfp4_b200", "csrc", name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
 
@@ -131,28 +133,48 @@ def max_over_ranks(v: float, ws: int) -> float:
 # ------------------------------------------------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms while the timed region runs.
+
+    The sampler is running (its first sample written) before the region starts.  Samples are matched to
+    the region by their timestamps; a region shorter than the sampling interval may hold none, and then
+    the samples just before and after it (same work, the warm-up and the steps after) stand in for it,
+    which the summary says."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    INTERVAL_MS = 50
 
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.INTERVAL_MS)],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (FileNotFoundError, OSError):
             self.proc = None
+        deadline = time.time() + 5.0
+        while self.proc is not None and time.time() < deadline and self.proc.poll() is None:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.01)
         return self
+
+    def start(self):
+        self.t0 = datetime.datetime.now()
+
+    def stop(self):
+        self.t1 = datetime.datetime.now()
 
     def __exit__(self, *exc):
         if self.proc is not None:
+            time.sleep(2 * self.INTERVAL_MS / 1000.0)  # one more sample after the region
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -162,27 +184,46 @@ class ClockSampler:
     def summary(self):
         if self.proc is None or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
-                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
-            except ValueError:
-                continue
+        with open(self.path) as fh:
+            lines = fh.readlines()
         os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        reasons = set()
-        for r in rows:
-            for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
-                            ("pcap", "sw_power_cap")):
-                if r[k].lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["smax"] for r in rows),
-                "power_w_max": max(r["power"] for r in rows), "samples": len(rows), "reasons": sorted(reasons)}
+        return summarize_clock_samples(lines, self.t0, self.t1)
+
+
+def summarize_clock_samples(lines, t0, t1):
+    """Median SM clock, max clock, max power and the throttle reasons seen in the samples taken between
+    t0 and t1 (datetimes), or in the nearest sample on each side when none falls in between."""
+    rows = []
+    for line in lines:
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 10:
+            continue
+        try:
+            rows.append(dict(t=datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f"), sm=float(parts[2]),
+                             smax=float(parts[3]), power=float(parts[4]), hw=parts[6], hwt=parts[7], swt=parts[8],
+                             pcap=parts[9]))
+        except ValueError:
+            continue
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+    window = "timed region"
+    if t0 is not None and t1 is not None:
+        inside = [r for r in rows if t0 <= r["t"] <= t1]
+        if not inside:
+            before = [r for r in rows if r["t"] < t0][-1:]
+            after = [r for r in rows if r["t"] > t1][:1]
+            inside = before + after
+            window = "adjacent to the timed region (shorter than the 50 ms sampling interval)"
+        rows = inside or rows
+    reasons = set()
+    for r in rows:
+        for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                        ("pcap", "sw_power_cap")):
+            if r[k].lower() == "active":
+                reasons.add(name)
+    return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["smax"] for r in rows),
+            "power_w_max": max(r["power"] for r in rows), "samples": len(rows), "window": window,
+            "reasons": sorted(reasons)}
 
 
 # ------------------------------------------------------------------------------------------
@@ -281,11 +322,13 @@ def run_native(args, ws, rank, local):
     barrier(ws)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
+        clk.start()
         start.record()
         for i in range(args.steps):
             bs.step({k: ev[k][i] for k in OPS})
         stop.record()
         torch.cuda.synchronize()
+        clk.stop()
     barrier(ws)
     B.check_device_error()
     ms_local = start.elapsed_time(stop)

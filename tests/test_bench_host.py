@@ -30,3 +30,30 @@ def test_traffic_follows_the_recorded_hash(monkeypatch, tmp_path):
     monkeypatch.setattr(bench, "TRAFFIC_PROFILE", str(p))
     monkeypatch.setattr(bench, "library_sources_sha256", lambda: "a" * 64)
     assert bench.measured_traffic() == 1234
+
+
+def _clock_line(t, sm, pcap="Not Active", hw="Not Active"):
+    return f"{t}, 0, {sm}, 1965, 600.5, 0x0, {hw}, Not Active, Not Active, {pcap}\n"
+
+
+def test_clock_samples_inside_the_timed_region():
+    import datetime
+    lines = [_clock_line("2026/12/02 10:00:00.000", 1200), _clock_line("2026/12/02 10:00:00.050", 1800, "Active"),
+             _clock_line("2026/12/02 10:00:00.100", 1700), _clock_line("2026/12/02 10:00:00.150", 900, hw="Active")]
+    t0 = datetime.datetime(2026, 12, 2, 10, 0, 0, 40000)
+    t1 = datetime.datetime(2026, 12, 2, 10, 0, 0, 120000)
+    s = bench.summarize_clock_samples(lines, t0, t1)
+    assert s["samples"] == 2 and s["sm_mhz"] == 1750 and s["reasons"] == ["sw_power_cap"]
+    assert s["window"] == "timed region"
+
+
+def test_clock_samples_adjacent_to_a_short_region():
+    import datetime
+    lines = [_clock_line("2026/12/02 10:00:00.000", 1500), _clock_line("2026/12/02 10:00:00.050", 1600),
+             _clock_line("2026/12/02 10:00:00.100", 1700, hw="Active")]
+    t0 = datetime.datetime(2026, 12, 2, 10, 0, 0, 60000)
+    t1 = datetime.datetime(2026, 12, 2, 10, 0, 0, 80000)
+    s = bench.summarize_clock_samples(lines, t0, t1)
+    assert s["samples"] == 2 and s["sm_mhz"] == 1650 and s["reasons"] == ["hw_slowdown"]
+    assert s["window"].startswith("adjacent")
+    assert bench.summarize_clock_samples(["garbage\n"], t0, t1)["reasons"] == ["no samples"]
