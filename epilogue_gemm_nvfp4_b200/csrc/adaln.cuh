@@ -8,15 +8,13 @@
 // FFN-up GEMM.  One warp owns one row at a time: the row's 16-element blocks are spread over the
 // lanes (lane l holds blocks l, l + 32, ...; 512 elements per warp step), the sum of squares is a
 // per-lane fp32 sum reduced by a butterfly (every lane ends with the same bits), and each lane then
-// modulates, rounds to bf16 and quantises its own blocks with the quantiser's block code.  Rows of up
-// to kAdalnSteps * 512 elements stay in registers between the two sweeps, so x is read from memory
-// once; longer rows are read again for the second sweep.
+// modulates, rounds to bf16 and quantises its own blocks with the quantiser's block code.
 //
-// Rows of up to kAdalnSteps * 512 elements take the staged form (kStaged): each warp owns a row buffer
-// in shared memory that a bulk copy (cp.async.bulk, counted on the warp's mbarrier) fills with its next
-// row while the warp computes the current one from registers, so the memory stream never waits for
-// the arithmetic.  Waits on the barrier are bounded; a wait that runs out sets the device error word
-// and the warp stops (after waiting, again bounded, for the copy it started).
+// The row is walked in chunks of kAdalnChunkSteps warp steps, twice: the first sweep streams it from
+// memory for the sum of squares, the second reads it again (from L2, where the first sweep just left
+// it) to modulate and quantise.  Holding a whole 4608-wide row in registers instead needs 124-167
+// registers per thread and leaves 12-16 warps per SM; the kernel is bound by dependent arithmetic
+// chains, not by memory, so it ran slower (81-86 us against 77 us for the [16896, 4608] tensor).
 //
 // With a dynamic tensor scale there are two launches of the same kernel: the amax pass computes u for
 // every row and reduces max |u| (its last CTA writes g), then the quantise pass recomputes u (the same
@@ -24,13 +22,11 @@
 // that its first rows are still in L2.
 #pragma once
 
-#include "gemm.cuh"
 #include "quantize.cuh"
 
 namespace nvfp4 {
 
-constexpr int kAdalnSteps = 9;          // 9 x 512 elements: a 4608-wide row held in registers
-constexpr int kAdalnStagedWarps = 4;    // warps per CTA of the staged form, one row buffer each
+constexpr int kAdalnChunkSteps = 2;  // warp steps (512 elements each) per chunk of a row
 
 struct AdalnArgs {
   const __nv_bfloat16* x;
@@ -52,14 +48,7 @@ struct AdalnArgs {
   // amax pass
   unsigned int* state;
   float* tensor_scale;
-  // staged form
-  int32_t row_buf_bytes;       // shared-memory bytes per warp's row buffer (2 * cols, rounded up to 128)
-  unsigned int* error_word;
-  uint64_t timeout_ns;
 };
-
-// Dynamic shared memory of the staged form: barriers and a zero flag, then one row buffer per warp.
-constexpr int kAdalnSmemHeader = 128;
 
 __device__ __forceinline__ void ld_mod16(const __nv_bfloat16* p, uint32_t (&v)[8]) {
   const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
@@ -90,12 +79,12 @@ __device__ __forceinline__ void modulate_block16(const uint32_t (&w)[8], float r
   }
 }
 
-// Steps [c0, c0 + kAdalnSteps) of a row into registers (zeros outside the row).
+// Steps [c0, c0 + kAdalnChunkSteps) of a row into registers (zeros outside the row).
 template <bool kVec32>
 __device__ __forceinline__ void ld_row_chunk(const __nv_bfloat16* xrow, int c0, int steps, int bpr, int lane,
-                                             uint32_t (&w)[kAdalnSteps][8]) {
+                                             uint32_t (&w)[kAdalnChunkSteps][8]) {
 #pragma unroll
-  for (int s = 0; s < kAdalnSteps; ++s) {
+  for (int s = 0; s < kAdalnChunkSteps; ++s) {
     const int blk = (c0 + s) * 32 + lane;
 #pragma unroll
     for (int i = 0; i < 8; ++i) w[s][i] = 0u;
@@ -103,94 +92,27 @@ __device__ __forceinline__ void ld_row_chunk(const __nv_bfloat16* xrow, int c0, 
   }
 }
 
-// Copy this lane's blocks of a row from the warp's shared-memory buffer into registers.
-__device__ __forceinline__ void ld_row_smem(const uint8_t* buf, int steps, int bpr, int lane,
-                                            uint32_t (&w)[kAdalnSteps][8]) {
-#pragma unroll
-  for (int s = 0; s < kAdalnSteps; ++s) {
-    const int blk = s * 32 + lane;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w[s][i] = 0u;
-    if (s < steps && blk < bpr) {
-      const uint4 lo = *reinterpret_cast<const uint4*>(buf + blk * 32);
-      const uint4 hi = *reinterpret_cast<const uint4*>(buf + blk * 32 + 16);
-      w[s][0] = lo.x; w[s][1] = lo.y; w[s][2] = lo.z; w[s][3] = lo.w;
-      w[s][4] = hi.x; w[s][5] = hi.y; w[s][6] = hi.z; w[s][7] = hi.w;
-    }
-  }
-}
-
-template <bool kAmaxPass, bool kReverse, bool kVec32, bool kStaged>
-__global__ void __launch_bounds__(kStaged ? 32 * kAdalnStagedWarps : 256, kStaged ? 3 : 2)
-    adaln_quantize_kernel(const AdalnArgs a) {
-  extern __shared__ __align__(128) uint8_t adaln_smem[];
+template <bool kAmaxPass, bool kReverse, bool kVec32>
+__global__ void __launch_bounds__(256, 4) adaln_quantize_kernel(const AdalnArgs a) {
   const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  const int64_t gwarp = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
+  const int64_t gwarp = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int bpr = static_cast<int>(a.cols / 16);
   const int steps = (bpr + 31) / 32;
-  const bool whole = steps <= kAdalnSteps;
   const float g = kAmaxPass ? 1.0f : *a.g_src;
   uint32_t umax = 0;  // amax pass: largest bf16 magnitude field of u seen by this lane
-
-  // staged form: this warp's barrier and row buffer; its first row's copy starts here
-  uint64_t* bar = reinterpret_cast<uint64_t*>(adaln_smem) + warp;
-  volatile int* never = reinterpret_cast<volatile int*>(adaln_smem + 64);  // stays 0: waits end on time only
-  uint8_t* buf = adaln_smem + kAdalnSmemHeader + warp * a.row_buf_bytes;
-  const uint32_t row_bytes = static_cast<uint32_t>(a.cols) * 2u;
-  uint32_t parity = 0;
-  bool pending = false;  // a copy into this warp's buffer has been started and not yet waited for
-  if constexpr (kStaged) {
-    if (threadIdx.x == 0) *never = 0;
-    if (lane == 0) {
-      mbar_init(bar, 1);
-      fence_mbarrier_init();
-    }
-    __syncthreads();
-    if (gwarp < a.rows) {
-      if (lane == 0) {
-        const int64_t row = kReverse ? a.rows - 1 - gwarp : gwarp;
-        mbar_arrive_expect_tx(bar, row_bytes);
-        bulk_load(buf, a.x + row * a.ldx, row_bytes, bar);
-      }
-      pending = true;
-    }
-  }
 
   for (int64_t t = gwarp; t < a.rows; t += nwarps) {
     const int64_t row = kReverse ? a.rows - 1 - t : t;
     const __nv_bfloat16* xrow = a.x + row * a.ldx;
-    uint32_t w[kAdalnSteps][8];
-
-    if constexpr (kStaged) {
-      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, never, a.timeout_ns));
-      if (!ok) {
-        if (lane == 0) atomicCAS(a.error_word, 0u, static_cast<unsigned int>(kErrTimeout));
-        break;
-      }
-      pending = false;
-      parity ^= 1u;
-      ld_row_smem(buf, steps, bpr, lane, w);
-      __syncwarp();
-      const int64_t tn = t + nwarps;  // this warp's next row goes into the buffer just read
-      if (tn < a.rows) {
-        if (lane == 0) {
-          const int64_t rn = kReverse ? a.rows - 1 - tn : tn;
-          fence_proxy_async_smem();
-          mbar_arrive_expect_tx(bar, row_bytes);
-          bulk_load(buf, a.x + rn * a.ldx, row_bytes, bar);
-        }
-        pending = true;
-      }
-    }
+    uint32_t w[kAdalnChunkSteps][8];
 
     // sweep 1: sum of squares (each square of a bf16 is exact in fp32)
     float ss = 0.0f;
-    for (int c0 = 0; c0 < steps; c0 += kAdalnSteps) {
-      if (!kStaged) ld_row_chunk<kVec32>(xrow, c0, steps, bpr, lane, w);
+    for (int c0 = 0; c0 < steps; c0 += kAdalnChunkSteps) {
+      ld_row_chunk<kVec32>(xrow, c0, steps, bpr, lane, w);
 #pragma unroll
-      for (int s = 0; s < kAdalnSteps; ++s) {
+      for (int s = 0; s < kAdalnChunkSteps; ++s) {
         float p = 0.0f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -215,11 +137,11 @@ __global__ void __launch_bounds__(kStaged ? 32 * kAdalnStagedWarps : 256, kStage
                               : a.scales + ((row >> 7) * a.k_atoms) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4;
     __nv_bfloat16* urow = (!kAmaxPass && a.u != nullptr) ? a.u + row * a.ld_u : nullptr;
 
-    // sweep 2: modulate, round to bf16, then reduce (amax pass) or quantise (a staged row is one chunk)
-    for (int c0 = 0; c0 < (kStaged ? 1 : steps); c0 += kAdalnSteps) {
-      if (!kStaged && !whole) ld_row_chunk<kVec32>(xrow, c0, steps, bpr, lane, w);
+    // sweep 2: modulate, round to bf16, then reduce (amax pass) or quantise
+    for (int c0 = 0; c0 < steps; c0 += kAdalnChunkSteps) {
+      ld_row_chunk<kVec32>(xrow, c0, steps, bpr, lane, w);
 #pragma unroll
-      for (int s = 0; s < kAdalnSteps; ++s) {
+      for (int s = 0; s < kAdalnChunkSteps; ++s) {
         if (c0 + s >= steps) break;  // warp-uniform
         const int blk = (c0 + s) * 32 + lane;
         const bool valid = blk < bpr;
@@ -241,11 +163,6 @@ __global__ void __launch_bounds__(kStaged ? 32 * kAdalnStagedWarps : 256, kStage
         }
       }
     }
-  }
-
-  if constexpr (kStaged) {
-    // a wait ran out: let the copy this warp started land before the CTA can exit
-    if (pending) (void)mbar_wait(bar, parity, never, a.timeout_ns);
   }
 
   if (kAmaxPass) {

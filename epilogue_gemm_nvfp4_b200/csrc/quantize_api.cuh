@@ -90,27 +90,14 @@ namespace {
 
 using AdalnKernel = void (*)(const AdalnArgs);
 
-AdalnKernel adaln_kernel_for(bool amax_pass, bool reverse, bool vec32, bool staged) {
-  if (staged) {
-    if (amax_pass) return adaln_quantize_kernel<true, false, false, true>;
-    return reverse ? adaln_quantize_kernel<false, true, false, true> : adaln_quantize_kernel<false, false, false, true>;
-  }
-  if (amax_pass) return vec32 ? adaln_quantize_kernel<true, false, true, false> : adaln_quantize_kernel<true, false, false, false>;
-  if (reverse) return vec32 ? adaln_quantize_kernel<false, true, true, false> : adaln_quantize_kernel<false, true, false, false>;
-  return vec32 ? adaln_quantize_kernel<false, false, true, false> : adaln_quantize_kernel<false, false, false, false>;
+AdalnKernel adaln_kernel_for(bool amax_pass, bool reverse, bool vec32) {
+  if (amax_pass) return vec32 ? adaln_quantize_kernel<true, false, true> : adaln_quantize_kernel<true, false, false>;
+  if (reverse) return vec32 ? adaln_quantize_kernel<false, true, true> : adaln_quantize_kernel<false, true, false>;
+  return vec32 ? adaln_quantize_kernel<false, false, true> : adaln_quantize_kernel<false, false, false>;
 }
 
-// One resident wave of CTAs (one row per warp at a time), at most as many warps as rows.
-int adaln_grid(AdalnKernel k, int threads, size_t smem, int64_t rows, int sm_count) {
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, smem) != cudaSuccess || per_sm < 1) per_sm = 1;
-  const int warps = threads / 32;
-  int64_t g = (rows + warps - 1) / warps;
-  const int64_t cap = static_cast<int64_t>(sm_count) * per_sm;
-  if (g > cap) g = cap;
-  if (g < 1) g = 1;
-  return static_cast<int>(g);
-}
+// One resident wave of 256-thread CTAs (one row per warp at a time), at most one warp per row.
+int adaln_grid(AdalnKernel k, int64_t rows, int sm_count) { return resident_grid(k, 256, rows, 8, sm_count); }
 
 }  // namespace
 
@@ -152,22 +139,15 @@ nvfp4_status nvfp4_adaln_quantize(const void* x, int64_t rows, int64_t cols, int
   a.u = static_cast<__nv_bfloat16*>(ada->u_out);
   a.ld_u = ada->ld_u;
   a.tensor_scale = out->tensor_scale;
-  a.error_word = st->error_word;
-  a.timeout_ns = wait_timeout_ns();
-  // rows that fit the registers stream through per-warp shared-memory buffers (the staged form)
-  const bool staged = (cols / 16 + 31) / 32 <= kAdalnSteps;
   const bool vec32 = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx * 2) % 32 == 0;
-  a.row_buf_bytes = staged ? static_cast<int32_t>((cols * 2 + 127) / 128 * 128) : 0;
-  const size_t smem = staged ? kAdalnSmemHeader + size_t(kAdalnStagedWarps) * a.row_buf_bytes : 0;
-  const int threads = staged ? 32 * kAdalnStagedWarps : 256;
   // dynamic scale: the amax pass walks the rows front to back, the quantise pass back to front
   if (compute_scale) {
     if (nvfp4_status e = amax_state_for(s, &a.state)) return e;
-    const AdalnKernel ak = adaln_kernel_for(true, false, vec32, staged);
-    ak<<<adaln_grid(ak, threads, smem, rows, st->sm_count), threads, smem, s>>>(a);
+    const AdalnKernel ak = adaln_kernel_for(true, false, vec32);
+    ak<<<adaln_grid(ak, rows, st->sm_count), 256, 0, s>>>(a);
   }
-  const AdalnKernel qk = adaln_kernel_for(false, compute_scale != 0, vec32, staged);
-  qk<<<adaln_grid(qk, threads, smem, rows + 1, st->sm_count), threads, smem, s>>>(a);
+  const AdalnKernel qk = adaln_kernel_for(false, compute_scale != 0, vec32);
+  qk<<<adaln_grid(qk, rows + 1, st->sm_count), 256, 0, s>>>(a);
   return launch_status();
 }
 

@@ -240,8 +240,8 @@ typedef struct {
  *                      nvfp4_quantize.
  *   compute_scale = 0: the g already stored in *out->tensor_scale is used; one launch.
  * Rules: cols % 16 == 0; x, ldx*2, shift, scale, ld_mod*2 (when read), u_out, ld_u*2, codes and scales
- * 16-byte aligned; rstd 4-byte aligned; ld_codes a multiple of 8.  Rows of up to 4608 elements are read
- * from memory once (twice with compute_scale = 1); longer rows once more per pass.
+ * 16-byte aligned; rstd 4-byte aligned; ld_codes a multiple of 8.  Each pass walks a row twice (sum of
+ * squares, then modulate and quantise); the second walk reads it from L2, so x crosses HBM once per pass.
  */
 NVFP4_API nvfp4_status nvfp4_adaln_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx,
                                             const nvfp4_adaln_desc* ada, int32_t compute_scale,
