@@ -48,14 +48,25 @@ TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "nvfp4_gemm_up_dram_2048sq.md")
 GEMM_SOURCES = ("ptx.cuh", "quantize.cuh", "gemm.cuh", "gemm_pair.cuh", "nvfp4_api.cu")
 
 
+def _code_only(text: str) -> str:
+    """Source text without // comments, trailing blanks and empty lines: a comment edit leaves it unchanged."""
+    lines = []
+    for line in text.splitlines():
+        code = line.split("//", 1)[0].rstrip()
+        if code:
+            lines.append(code)
+    return "\n".join(lines)
+
+
 def library_sources_sha256():
-    """sha256 over the up GEMM's sources (GEMM_SOURCES: file name, then bytes, in that order)."""
+    """sha256 over the code of the up GEMM's sources (GEMM_SOURCES, comments dropped): each file's name,
+    then its code, in that order."""
     import hashlib
     h = hashlib.sha256()
     for name in GEMM_SOURCES:
         h.update(name.encode())
-        with open(os.path.join(ROOT, "epilogue_gemm_nvfp4_b200", "csrc", name), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "epilogue_gemm_nvfp4_b200", "csrc", name)) as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()
 
 

@@ -22,8 +22,8 @@
 //                 requantisation from registers.  Row-wise reductions stay within the two threads that
 //                 hold a row: for the 256-wide head each adds the squares of its 128 columns and the
 //                 two partial sums meet in shared memory, so the head is never revisited.
-//                 Stores go through a 1 KB per-warp shared-memory transpose so that each st.global
-//                 writes whole 32-byte row segments.
+//                 Each warp writes its 32 rows of a 16- or 32-column slice into its own shared-memory
+//                 box in the TMA swizzle, and one lane hands the box to a TMA bulk tensor store.
 // The per-stage TMEM scale slot is safe to rewrite without extra waits: the producer refills stage s
 // only after the commit of the MMAs that read stage s.
 #pragma once

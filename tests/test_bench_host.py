@@ -57,3 +57,9 @@ def test_clock_samples_adjacent_to_a_short_region():
     assert s["samples"] == 2 and s["sm_mhz"] == 1650 and s["reasons"] == ["hw_slowdown"]
     assert s["window"].startswith("adjacent")
     assert bench.summarize_clock_samples(["garbage\n"], t0, t1)["reasons"] == ["no samples"]
+
+
+def test_traffic_hash_ignores_comments_only():
+    code = "int a = 1;  // one\n\n// a note\nint b = 2;\n"
+    assert bench._code_only(code) == bench._code_only("int a = 1;  // changed\nint b = 2;   \n")
+    assert bench._code_only(code) != bench._code_only("int a = 1;\nint b = 3;\n")
