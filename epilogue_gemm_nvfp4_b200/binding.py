@@ -202,10 +202,18 @@ def adaln_quantize(x: torch.Tensor, shift: torch.Tensor | None = None, scale: to
     compute = g is None and not static
     mods = [m for m in (shift, scale) if m is not None]
     for m in mods:
-        assert m.is_cuda and m.dtype == torch.bfloat16 and m.stride(-1) == 1
-    ld_mod = mods[0].stride(0) if mods and mods[0].dim() == 2 else cols
-    if len(mods) == 2 and mods[0].dim() == 2:
-        assert mods[1].dim() == 2 and mods[1].stride(0) == ld_mod, "shift and scale need the same sample stride"
+        assert m.is_cuda and m.dtype == torch.bfloat16 and m.stride(-1) == 1 and m.shape[-1] == cols
+    samples = 1 if rows_per_sample <= 0 or rows_per_sample >= rows else -(-rows // rows_per_sample)
+    ld_mod = cols
+    if mods:
+        dims = {m.dim() for m in mods}
+        assert dims in ({1}, {2}), "shift and scale are both [cols] or both [samples, cols]"
+        if dims == {2}:
+            ld_mod = mods[0].stride(0)
+            assert all(m.stride(0) == ld_mod and m.shape[0] >= samples for m in mods), \
+                "shift and scale need the same sample stride and one row per sample"
+        else:
+            assert samples == 1, "per-sample modulation needs [samples, cols] vectors"
     desc = CAdaln(_ptr(shift), _ptr(scale), int(ld_mod), int(rows_per_sample), float(eps), _ptr(rstd),
                   _ptr(u_out), u_out.stride(0) if u_out is not None else 0)
     ct = out.c()
