@@ -575,3 +575,37 @@ def test_w8a8_error_bound():
     bound = (np.abs(x).astype(np.float64) @ np.ones((64, 8))) * ew.T + ex * (np.ones((6, 64)) @ np.abs(w).T) \
         + 64 * ex * ew.T
     assert np.all(np.abs(y - x.astype(np.float64) @ w.astype(np.float64).T) <= bound * (1 + 1e-6))
+
+
+def test_adaln_is_equivariant_to_column_permutations():
+    """RMSNorm and a per-column modulation commute with any permutation of the columns."""
+    rng = np.random.default_rng(14)
+    x = rng.standard_normal((6, 48))
+    sh, sc = rng.standard_normal(48), rng.standard_normal(48)
+    p = rng.permutation(48)
+    u, r = O.adaln_modulate(x, sh, sc)
+    up, rp = O.adaln_modulate(x[:, p], sh[p], sc[p])
+    np.testing.assert_allclose(up, u[:, p], rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(rp, r, rtol=1e-14)
+
+
+def test_int8_rows_scale_by_powers_of_two():
+    """Multiplying a row by 2^k leaves its codes unchanged and multiplies its scale by 2^k exactly."""
+    rng = np.random.default_rng(15)
+    x = rng.standard_normal((5, 64)).astype(np.float32)
+    q, s = O.int8_quantize_rows(x)
+    for k in (-7, 3, 20):
+        q2, s2 = O.int8_quantize_rows(x * np.float32(2.0 ** k))
+        assert np.array_equal(q2, q)
+        assert np.array_equal(s2, (s * np.float32(2.0 ** k)).astype(np.float32))
+
+
+def test_quantize_scales_by_powers_of_two_with_the_tensor():
+    """NVFP4 of 2^k x has the codes and block scales of x and a tensor scale 2^k times larger."""
+    rng = np.random.default_rng(16)
+    x = rng.standard_normal((4, 64)).astype(np.float32)
+    c, s, g = O.quantize(x)
+    for k in (-5, 4):
+        c2, s2, g2 = O.quantize(x * np.float32(2.0 ** k))
+        assert np.array_equal(c2, c) and np.array_equal(s2, s)
+        assert g2 == np.float32(g * np.float32(2.0 ** k))
