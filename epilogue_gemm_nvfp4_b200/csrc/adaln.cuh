@@ -13,8 +13,8 @@
 // The row is walked in chunks of kAdalnChunkSteps warp steps, twice: the first sweep streams it from
 // memory for the sum of squares, the second reads it again (from L2, where the first sweep just left
 // it) to modulate and quantise.  Holding a whole 4608-wide row in registers instead needs 124-167
-// registers per thread and leaves 12-16 warps per SM; the kernel is bound by dependent arithmetic
-// chains, not by memory, so it ran slower (81-86 us against 77 us for the [16896, 4608] tensor).
+// registers per thread and leaves 12-16 warps per SM; the kernel is bound by instruction issue and
+// dependent arithmetic, not by memory, so it ran slower (81-86 us against 77 us for [16896, 4608]).
 //
 // With a dynamic tensor scale there are two launches of the same kernel: the amax pass computes u for
 // every row and reduces max |u| (its last CTA writes g), then the quantise pass recomputes u (the same
