@@ -160,3 +160,39 @@ def test_ctypes_structs_match_the_header(tmp_path):
         assert got[(cname, "size")] == ctypes.sizeof(py), cname
         for field, _ in py._fields_:
             assert got[(cname, field)] == getattr(py, field).offset, (cname, field)
+
+
+def test_c_program_links_and_calls_the_abi(tmp_path):
+    """A plain C program, compiled with gcc against include/nvfp4.h and linked with libnvfp4.so, calls the
+    host helpers and gets the documented argument errors (no device needed)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    lib_dir = os.path.dirname(B.LIB_PATH)
+    src = tmp_path / "use.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "nvfp4.h"
+int main(void) {
+  nvfp4_tensor t = {(void*)0x10000, (void*)0x10000, (float*)0x10000, 4, 520, 0};
+  nvfp4_epilogue_desc epi = {0};
+  nvfp4_tensor a = {(void*)0x10000, (void*)0x10000, (float*)0x10000, 256, 512, 0};
+  nvfp4_tensor w = {(void*)0x10000, (void*)0x10000, (float*)0x10000, 200, 512, 0};
+  printf("%zu %lld %d %d %d %s\n", nvfp4_scale_bytes(300, 208), (long long)nvfp4_scale_offset(130, 5, 208),
+         (int)nvfp4_quantize((void*)0x10000, 4, 520, 520, 1, &t, NULL),
+         (int)nvfp4_linear(&a, &w, &epi, (void*)0x10000, 512, NULL, NULL),
+         (int)nvfp4_linear_tile_n(13824, 4608, NVFP4_EPI_QKNORM), nvfp4_status_string(NVFP4_ERR_MISALIGNED));
+  return 0;
+}
+''')
+    exe = tmp_path / "use"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe), "-L", lib_dir,
+                    "-lnvfp4", f"-Wl,-rpath,{lib_dir}"], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert int(out[0]) == O.scale_buffer_bytes(300, 208)
+    assert int(out[1]) == O.scale_atom_offset(130, 5, 208)
+    assert int(out[2]) == B.ERR_UNSUPPORTED_SHAPE          # cols % 16
+    assert int(out[3]) == B.ERR_UNSUPPORTED_SHAPE          # N % 128
+    assert int(out[4]) == 256
+    assert " ".join(out[5:]).startswith("misaligned")
