@@ -84,7 +84,7 @@ __device__ __forceinline__ void modulate_block16(const uint32_t (&w)[8], float r
 // columns, in fp32.  A warp step's read of one word index is 32 consecutive 16-byte entries, so the
 // reads are free of bank conflicts, and the per-element unpacking and the 1 + scale add happen once
 // per CTA instead of once per row.
-constexpr int kAdalnTableMaxSteps = 12;  // up to 6144 columns: 48 KB of table per CTA
+constexpr int kAdalnTableMaxSteps = 11;  // up to 5632 columns: 44 KB of table, under the 48 KB default with the static reduction buffer
 
 __device__ __forceinline__ int adaln_table_index(int col) {
   const int blk = col >> 4, i = (col & 15) >> 1;

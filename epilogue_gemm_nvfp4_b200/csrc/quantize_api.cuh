@@ -154,7 +154,7 @@ nvfp4_status nvfp4_adaln_quantize(const void* x, int64_t rows, int64_t cols, int
   a.ld_u = ada->ld_u;
   a.tensor_scale = out->tensor_scale;
   const bool vec32 = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx * 2) % 32 == 0;
-  // one sample and rows of at most 6144 elements: the modulation comes from a shared-memory table
+  // one sample and rows of at most 5632 elements: the modulation comes from a shared-memory table
   const int64_t steps = (cols / 16 + 31) / 32;
   const bool table = a.rows_per_sample == 0 && steps <= kAdalnTableMaxSteps;
   const size_t smem = table ? static_cast<size_t>(steps) * 8 * 32 * sizeof(float4) : 0;
