@@ -79,6 +79,48 @@ __device__ __forceinline__ void modulate_block16(const uint32_t (&w)[8], float r
   }
 }
 
+// The modulation of a single sample as a shared-memory table: for bf16x2 word i of the block a lane
+// holds in warp step st, entry (st * 8 + i) * 32 + lane is {1 + scale, shift} of the word's two
+// columns, in fp32.  A warp step's read of one word index is 32 consecutive 16-byte entries, so the
+// reads are free of bank conflicts, and the per-element unpacking and the 1 + scale add happen once
+// per CTA instead of once per row.
+constexpr int kAdalnTableMaxSteps = 11;  // up to 5632 columns: 44 KB of table, under the 48 KB default with the static reduction buffer
+
+__device__ __forceinline__ int adaln_table_index(int col) {
+  const int blk = col >> 4, i = (col & 15) >> 1;
+  return ((blk >> 5) * 8 + i) * 32 + (blk & 31);
+}
+
+__device__ void fill_adaln_table(float4* tab, const AdalnArgs& a) {
+  for (int c = 2 * static_cast<int>(threadIdx.x); c < a.cols; c += 2 * static_cast<int>(blockDim.x)) {
+    float m0 = 1.0f, m1 = 1.0f, s0 = 0.0f, s1 = 0.0f;
+    if (a.scale) {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(a.scale + c);
+      m0 = __fadd_rn(1.0f, __uint_as_float(w << 16));
+      m1 = __fadd_rn(1.0f, __uint_as_float(w & 0xFFFF0000u));
+    }
+    if (a.shift) {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(a.shift + c);
+      s0 = __uint_as_float(w << 16);
+      s1 = __uint_as_float(w & 0xFFFF0000u);
+    }
+    tab[adaln_table_index(c)] = make_float4(m0, s0, m1, s1);
+  }
+}
+
+// modulate_block16 from the table (the same operations on the same fp32 values, so the same bits).
+__device__ __forceinline__ void modulate_block16_tab(const uint32_t (&w)[8], float rstd, const float4* tab, int st,
+                                                     int lane, uint32_t (&u)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 t = tab[(st * 8 + i) * 32 + lane];
+    const float lo = __fmaf_rn(__fmul_rn(__uint_as_float(w[i] << 16), rstd), t.x, t.y);
+    const float hi = __fmaf_rn(__fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), rstd), t.z, t.w);
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    u[i] = *reinterpret_cast<const uint32_t*>(&p);
+  }
+}
+
 // Steps [c0, c0 + kAdalnChunkSteps) of a row into registers (zeros outside the row).
 template <bool kVec32>
 __device__ __forceinline__ void ld_row_chunk(const __nv_bfloat16* xrow, int c0, int steps, int bpr, int lane,
@@ -92,8 +134,15 @@ __device__ __forceinline__ void ld_row_chunk(const __nv_bfloat16* xrow, int c0, 
   }
 }
 
-template <bool kAmaxPass, bool kReverse, bool kVec32>
+// kTable: one sample for every row and at most kAdalnTableMaxSteps warp steps per row; the modulation
+// then comes from the shared-memory table (dynamic shared memory of steps * 4 KB).
+template <bool kAmaxPass, bool kReverse, bool kVec32, bool kTable>
 __global__ void __launch_bounds__(256, 4) adaln_quantize_kernel(const AdalnArgs a) {
+  extern __shared__ float4 adaln_tab[];
+  if constexpr (kTable) {
+    fill_adaln_table(adaln_tab, a);
+    __syncthreads();
+  }
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   const int64_t gwarp = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -148,8 +197,12 @@ __global__ void __launch_bounds__(256, 4) adaln_quantize_kernel(const AdalnArgs 
         uint32_t u[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) u[i] = 0u;
-        if (valid)
-          modulate_block16(w[s], rstd, shrow ? shrow + blk * 16 : nullptr, scrow ? scrow + blk * 16 : nullptr, u);
+        if (valid) {
+          if constexpr (kTable)
+            modulate_block16_tab(w[s], rstd, adaln_tab, c0 + s, lane, u);
+          else
+            modulate_block16(w[s], rstd, shrow ? shrow + blk * 16 : nullptr, scrow ? scrow + blk * 16 : nullptr, u);
+        }
         if (kAmaxPass) {
 #pragma unroll
           for (int i = 0; i < 8; ++i) umax = max(umax, max(u[i] & 0x7FFFu, (u[i] >> 16) & 0x7FFFu));

@@ -90,14 +90,28 @@ namespace {
 
 using AdalnKernel = void (*)(const AdalnArgs);
 
-AdalnKernel adaln_kernel_for(bool amax_pass, bool reverse, bool vec32) {
-  if (amax_pass) return vec32 ? adaln_quantize_kernel<true, false, true> : adaln_quantize_kernel<true, false, false>;
-  if (reverse) return vec32 ? adaln_quantize_kernel<false, true, true> : adaln_quantize_kernel<false, true, false>;
-  return vec32 ? adaln_quantize_kernel<false, false, true> : adaln_quantize_kernel<false, false, false>;
+AdalnKernel adaln_kernel_for(bool amax_pass, bool reverse, bool vec32, bool table) {
+#define NVFP4_ADALN_PICK(T)                                                                                   \
+  if (amax_pass) return vec32 ? adaln_quantize_kernel<true, false, true, T> : adaln_quantize_kernel<true, false, false, T>; \
+  if (reverse) return vec32 ? adaln_quantize_kernel<false, true, true, T> : adaln_quantize_kernel<false, true, false, T>;    \
+  return vec32 ? adaln_quantize_kernel<false, false, true, T> : adaln_quantize_kernel<false, false, false, T>;
+  if (table) {
+    NVFP4_ADALN_PICK(true)
+  }
+  NVFP4_ADALN_PICK(false)
+#undef NVFP4_ADALN_PICK
 }
 
 // One resident wave of 256-thread CTAs (one row per warp at a time), at most one warp per row.
-int adaln_grid(AdalnKernel k, int64_t rows, int sm_count) { return resident_grid(k, 256, rows, 8, sm_count); }
+int adaln_grid(AdalnKernel k, size_t smem, int64_t rows, int sm_count) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, 256, smem) != cudaSuccess || per_sm < 1) per_sm = 1;
+  int64_t g = (rows + 7) / 8;
+  const int64_t cap = static_cast<int64_t>(sm_count) * per_sm;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return static_cast<int>(g);
+}
 
 }  // namespace
 
@@ -140,14 +154,18 @@ nvfp4_status nvfp4_adaln_quantize(const void* x, int64_t rows, int64_t cols, int
   a.ld_u = ada->ld_u;
   a.tensor_scale = out->tensor_scale;
   const bool vec32 = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx * 2) % 32 == 0;
+  // one sample and rows of at most 5632 elements: the modulation comes from a shared-memory table
+  const int64_t steps = (cols / 16 + 31) / 32;
+  const bool table = a.rows_per_sample == 0 && steps <= kAdalnTableMaxSteps;
+  const size_t smem = table ? static_cast<size_t>(steps) * 8 * 32 * sizeof(float4) : 0;
   // dynamic scale: the amax pass walks the rows front to back, the quantise pass back to front
   if (compute_scale) {
     if (nvfp4_status e = amax_state_for(s, &a.state)) return e;
-    const AdalnKernel ak = adaln_kernel_for(true, false, vec32);
-    ak<<<adaln_grid(ak, rows, st->sm_count), 256, 0, s>>>(a);
+    const AdalnKernel ak = adaln_kernel_for(true, false, vec32, table);
+    ak<<<adaln_grid(ak, smem, rows, st->sm_count), 256, smem, s>>>(a);
   }
-  const AdalnKernel qk = adaln_kernel_for(false, compute_scale != 0, vec32);
-  qk<<<adaln_grid(qk, rows + 1, st->sm_count), 256, 0, s>>>(a);
+  const AdalnKernel qk = adaln_kernel_for(false, compute_scale != 0, vec32, table);
+  qk<<<adaln_grid(qk, smem, rows + 1, st->sm_count), 256, smem, s>>>(a);
   return launch_status();
 }
 
