@@ -556,6 +556,32 @@ def op_case(name):
         scale = torch.full((1,), 3.0 / 2688.0, dtype=torch.float32, device=dev)
         return (lambda: B.fake_quantize(x, y=y, scale=scale, static=static)), 4.0 * rows * cols, "GB/s (4 B/elem)"
 
+    def gemm_i8(case, requant=False):
+        a = B.int8_quantize(case.x.to(dev))
+        w = B.int8_quantize(case.w.to(dev))
+        bias = case.bias.to(dev) if case.bias is not None else None
+        ex = {}
+        if case.epilogue == "qknorm":
+            e = case.extras
+            ex = dict(gamma_q=e["gamma_q"].to(dev), gamma_k=e["gamma_k"].to(dev), eps=e["eps"], q_col0=e["q_col0"],
+                      k_col0=e["k_col0"], qk_cols=e["qk_cols"], head_dim=e["head_dim"])
+        elif case.epilogue == "resid_gate":
+            ex = dict(residual=case.extras["residual"].to(dev), gate=case.extras["gate"].to(dev))
+        q = None
+        if requant:
+            q = B.QTensor.empty(case.M, case.n_out)
+            q.g.fill_(0.01)
+        out = torch.empty(case.M, case.n_out, dtype=torch.bfloat16, device=dev)
+        fn = lambda: B.int8_linear(a, w, case.epilogue, bias=bias, out=out if q is None else None, out_fp4=q,
+                                   want_bf16=q is None, **ex)
+        return fn, W.flops(case), "TOP/s (int8)"
+
+    def int8_quant(rows, cols):
+        x = W.to_bf16(W.normal(np.random.default_rng(0), (rows, cols))).to(dev)
+        mult = torch.rand(cols, dtype=torch.float32, device=dev) + 0.5
+        out = B.Int8Tensor.empty(rows, cols)
+        return (lambda: B.int8_quantize(x, mult, out=out)), 3.0 * rows * cols + 4.0 * (rows + cols), "GB/s (3 B/elem)"
+
     def adaln(static=False):
         case = W.adaln_2k()
         x, sh, sc = case.x.to(dev), case.shift[0].to(dev), case.scale[0].to(dev)
@@ -590,6 +616,11 @@ def op_case(name):
         "fakeq_2k_static": lambda: fakeq(M2, W.HIDDEN, static=True),
         "quant_text_static": lambda: quant(W.HIDDEN, W.TEXT_K, static=True),
         "amax_2k": lambda: amax(M2, W.HIDDEN),
+        "w8a8_qkv_1k": lambda: gemm_i8(W.qkv_1k()),
+        "w8a8_up_1k": lambda: gemm_i8(W.case_ffn_up(M1), requant=True),
+        "w8a8_down_1k": lambda: gemm_i8(W.case_ffn_down(M1)),
+        "w8a8_out_2k": lambda: gemm_i8(W.case_bias(M2, W.HIDDEN, W.HIDDEN, seed=8, w_std=0.015)),
+        "int8_quant_2k": lambda: int8_quant(M2, W.HIDDEN),
         "adaln_2k": lambda: adaln(),
         "adaln_2k_static": lambda: adaln(static=True),
     }
@@ -617,7 +648,7 @@ def run_op(args):
         reps.append(s.elapsed_time(e) / args.steps)
     B.check_device_error()
     med = sorted(reps)[1]
-    scale = 1e12 if unit.startswith("TFLOP") else 1e9
+    scale = 1e12 if unit.startswith(("TFLOP", "TOP")) else 1e9
     return {"op": args.op, "mean_us": round(med * 1e3, 2), "min_us": round(min(reps) * 1e3, 2),
             "value": round(work / (med * 1e-3) / scale, 1), "unit": unit, "steps": args.steps}
 

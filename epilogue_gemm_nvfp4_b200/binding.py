@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libnvfp4.so")
 EXPORTS = ("nvfp4_quantize", "nvfp4_linear", "nvfp4_dequantize", "nvfp4_amax", "nvfp4_scale_bytes",
            "nvfp4_scale_offset", "nvfp4_get_device_error", "nvfp4_linear_tile_n", "nvfp4_linear_split_k",
            "nvfp4_status_string", "nvfp4_version", "nvfp4_linear_noalloc", "nvfp4_linear_noalloc_scratch_bytes",
-           "nvfp4_fake_quantize", "nvfp4_adaln_quantize")
+           "nvfp4_fake_quantize", "nvfp4_adaln_quantize", "nvfp4_int8_quantize", "nvfp4_int8_linear")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_MISALIGNED, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_SCRATCH_LIMIT = range(7)
 EPI_BIAS, EPI_QKNORM, EPI_GATED_SILU, EPI_RESID_GATE = range(4)
@@ -46,6 +46,11 @@ class CAdaln(ctypes.Structure):
                 ("u_out", ctypes.c_void_p), ("ld_u", ctypes.c_int64)]
 
 
+class CInt8Tensor(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("ld", ctypes.c_int64)]
+
+
 class NvFp4Error(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
@@ -67,6 +72,7 @@ def load() -> ctypes.CDLL:
     TP = ctypes.POINTER(CTensor)
     EP = ctypes.POINTER(CEpilogue)
     AP = ctypes.POINTER(CAdaln)
+    IP = ctypes.POINTER(CInt8Tensor)
     sig = {
         "nvfp4_quantize": (I32, [P, I64, I64, I64, I32, TP, P]),
         "nvfp4_linear": (I32, [TP, TP, EP, P, I64, TP, P]),
@@ -75,6 +81,8 @@ def load() -> ctypes.CDLL:
         "nvfp4_dequantize": (I32, [TP, P, I64, P]),
         "nvfp4_fake_quantize": (I32, [P, I64, I64, I64, I32, P, P, I64, P]),
         "nvfp4_adaln_quantize": (I32, [P, I64, I64, I64, AP, I32, TP, P]),
+        "nvfp4_int8_quantize": (I32, [P, I64, I64, I64, P, IP, P]),
+        "nvfp4_int8_linear": (I32, [IP, IP, EP, P, I64, TP, P]),
         "nvfp4_amax": (I32, [P, I64, I64, I64, P, P]),
         "nvfp4_scale_bytes": (SZ, [I64, I64]),
         "nvfp4_scale_offset": (I64, [I64, I64, I64]),
@@ -259,6 +267,58 @@ def linear(a: QTensor, w: QTensor, kind: str = "bias", bias=None, out: torch.Ten
     _check(load().nvfp4_linear(ctypes.byref(ca), ctypes.byref(cw), ctypes.byref(desc), _ptr(out),
                                out.stride(0) if out is not None else 0,
                                ctypes.byref(cq) if cq is not None else None, _stream(stream)), "nvfp4_linear")
+    return out
+
+
+# ------------------------------------------------------------------------------------------
+# W8A8 INT8 path
+# ------------------------------------------------------------------------------------------
+
+@dataclass
+class Int8Tensor:
+    """Per-row INT8: codes int8 [rows, cols] and the fp32 decode scale of each row [rows]."""
+    q: torch.Tensor
+    scale: torch.Tensor
+    rows: int
+    cols: int
+
+    @classmethod
+    def empty(cls, rows: int, cols: int, device="cuda") -> "Int8Tensor":
+        return cls(torch.empty((rows, cols), dtype=torch.int8, device=device),
+                   torch.empty(max(rows, 1), dtype=torch.float32, device=device), rows, cols)
+
+    def c(self) -> CInt8Tensor:
+        return CInt8Tensor(self.q.data_ptr(), self.scale.data_ptr(), self.rows, self.cols, self.q.stride(0))
+
+
+def int8_quantize(x: torch.Tensor, col_mult: torch.Tensor | None = None, out: Int8Tensor | None = None,
+                  stream=None) -> Int8Tensor:
+    """bf16 [rows, cols] -> per-row INT8 through nvfp4_int8_quantize; ``col_mult`` (fp32 [cols]) multiplies
+    each column first (1 / lambda for activations, lambda for a weight under SmoothQuant)."""
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    if col_mult is not None:
+        assert col_mult.is_cuda and col_mult.dtype == torch.float32 and col_mult.numel() == cols
+    out = Int8Tensor.empty(rows, cols, x.device) if out is None else out
+    ct = out.c()
+    _check(load().nvfp4_int8_quantize(_ptr(x), rows, cols, x.stride(0), _ptr(col_mult), ctypes.byref(ct),
+                                      _stream(stream)), "nvfp4_int8_quantize")
+    return out
+
+
+def int8_linear(a: Int8Tensor, w: Int8Tensor, kind: str = "bias", bias=None, out: torch.Tensor | None = None,
+                out_fp4: QTensor | None = None, want_bf16: bool = True, stream=None, **epi) -> torch.Tensor | None:
+    """Fused W8A8 linear through nvfp4_int8_linear (the epilogue arguments of ``linear``)."""
+    n_out = w.rows // 2 if kind == "gated_silu" else w.rows
+    if out is None and want_bf16:
+        out = torch.empty((a.rows, n_out), dtype=torch.bfloat16, device=a.q.device)
+    desc = make_epilogue(kind, bias=bias, out_nvfp4=out_fp4 is not None, **epi)
+    ca, cw = a.c(), w.c()
+    cq = out_fp4.c() if out_fp4 is not None else None
+    _check(load().nvfp4_int8_linear(ctypes.byref(ca), ctypes.byref(cw), ctypes.byref(desc), _ptr(out),
+                                    out.stride(0) if out is not None else 0,
+                                    ctypes.byref(cq) if cq is not None else None, _stream(stream)),
+           "nvfp4_int8_linear")
     return out
 
 

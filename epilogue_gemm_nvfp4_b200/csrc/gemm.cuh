@@ -71,6 +71,8 @@ struct GemmArgs {
   const float* q_g;
   int32_t q_k_atoms;
   unsigned int* out_amax_bits;  // raised to max |bf16 output| (fp32 bit pattern), or nullptr
+  const float* row_scale;       // INT8 form: decode scale of each row of A [M]
+  const float* col_scale;       // INT8 form: decode scale of each row of W [N]
   unsigned int* error_word;
   uint64_t timeout_ns;
   // split-K: `splits` consecutive work units share one output tile, each summing a contiguous range
@@ -96,7 +98,9 @@ __device__ __forceinline__ WorkUnit work_unit(const GemmArgs& a, int u, int num_
   return w;
 }
 
-template <int BN>
+// kI8: the W8A8 INT8 form of the same kernel (tcgen05.mma.kind::i8, s32 accumulators): no block
+// scales to stage, so no scale slots in shared memory or TMEM, and two accumulators even at BN = 256.
+template <int BN, bool kI8 = false>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int THREADS = 512;
@@ -105,13 +109,13 @@ struct GemmCfg {
   static constexpr int A_BYTES = BM * BK_BYTES;
   static constexpr int B_BYTES = BN * BK_BYTES;
   static constexpr int SF_ATOM_BYTES = 512;             // 128 rows x 4 blocks
-  static constexpr int SFA_BYTES = KSTEPS * SF_ATOM_BYTES;
-  static constexpr int SFB_BYTES = (BN / 128) * KSTEPS * SF_ATOM_BYTES;
+  static constexpr int SFA_BYTES = kI8 ? 0 : KSTEPS * SF_ATOM_BYTES;
+  static constexpr int SFB_BYTES = kI8 ? 0 : (BN / 128) * KSTEPS * SF_ATOM_BYTES;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int ACC_BUFS = BN == 256 ? 1 : 2;
+  static constexpr int ACC_BUFS = (BN == 256 && !kI8) ? 1 : 2;
   static constexpr int SF_COL0 = ACC_BUFS * BN;         // TMEM columns after the accumulator(s)
-  static constexpr int SFA_COLS = KSTEPS * 4;
-  static constexpr int SFB_COLS = KSTEPS * (BN / 32);
+  static constexpr int SFA_COLS = kI8 ? 0 : KSTEPS * 4;
+  static constexpr int SFB_COLS = kI8 ? 0 : KSTEPS * (BN / 32);
   static constexpr int SF_COLS = SFA_COLS + SFB_COLS;
   static constexpr int TMEM_COLS = 512;
   static constexpr int EPI_WARPS = 8;
@@ -121,10 +125,10 @@ struct GemmCfg {
   static constexpr int SMEM_LIMIT = 232448;
   // as many stages as shared memory and the TMEM scale slots allow
   static constexpr int STAGES_SMEM = (SMEM_LIMIT - AUX_BYTES - 1023 - EPI_WARPS * XPOSE_BYTES) / STAGE_BYTES;
-  static constexpr int STAGES_TMEM = (TMEM_COLS - SF_COL0) / SF_COLS;
+  static constexpr int STAGES_TMEM = kI8 ? STAGES_SMEM : (TMEM_COLS - SF_COL0) / (SF_COLS > 0 ? SF_COLS : 1);
   static constexpr int STAGES = STAGES_SMEM < STAGES_TMEM ? STAGES_SMEM : STAGES_TMEM;
   static constexpr int SMEM_BYTES = AUX_BYTES + 1023 + STAGES * STAGE_BYTES + EPI_WARPS * XPOSE_BYTES;
-  static constexpr uint32_t IDESC = idesc_nvf4(BM, BN);
+  static constexpr uint32_t IDESC = kI8 ? idesc_i8(BM, BN) : idesc_nvf4(BM, BN);
   static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(SF_COLS % 8 == 0, "scale slot is written 8 columns at a time");
   static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
@@ -431,6 +435,35 @@ struct Epilogue {
   }
 };
 
+// INT8 form: the accumulator columns hold s32 sums (their bits, as loaded); turn each into fp32 and
+// multiply it by its weight row's decode scale.  The row's activation scale enters as the epilogue's
+// alpha.  Columns of the gated SiLU: this thread's 64 a columns, then the matching 64 b columns.
+template <int BN, int KIND>
+__device__ __forceinline__ void i8_scale_columns(const GemmArgs& a, int e, int nb, float* acc) {
+  auto scale32 = [&](float* v, int col0) {
+    const float4* cs = reinterpret_cast<const float4*>(a.col_scale + col0);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 c = __ldg(cs + q);
+      v[4 * q + 0] = __fmul_rn(__int2float_rn(__float_as_int(v[4 * q + 0])), c.x);
+      v[4 * q + 1] = __fmul_rn(__int2float_rn(__float_as_int(v[4 * q + 1])), c.y);
+      v[4 * q + 2] = __fmul_rn(__int2float_rn(__float_as_int(v[4 * q + 2])), c.z);
+      v[4 * q + 3] = __fmul_rn(__int2float_rn(__float_as_int(v[4 * q + 3])), c.w);
+    }
+  };
+  if constexpr (KIND == kEpiGatedSilu) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      scale32(acc + 32 * c, nb * 128 + 64 * e + 32 * c);
+      scale32(acc + 64 + 32 * c, a.N / 2 + nb * 128 + 64 * e + 32 * c);
+    }
+  } else {
+    constexpr int COLS = Epilogue<BN, KIND>::COLS;
+#pragma unroll
+    for (int c = 0; c < COLS / 32; ++c) scale32(acc + 32 * c, nb * BN + COLS * e + 32 * c);
+  }
+}
+
 constexpr unsigned int kSplitReady = 0x100u;
 
 // Split-K hand-off for one tile (two work units).  Returns true when this CTA now holds the full sum
@@ -481,11 +514,11 @@ __device__ __forceinline__ bool split_exchange(const GemmArgs& a, int tile, int 
   return true;
 }
 
-template <int BN, int KIND>
+template <int BN, int KIND, bool kI8 = false>
 __global__ void __launch_bounds__(512, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ OutMaps out_maps, const __grid_constant__ GemmArgs args) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, kI8>;
   using E = Epilogue<BN, KIND>;
   extern __shared__ uint8_t smem_raw[];
   // small state first, then the 1024-aligned stage ring (128-byte swizzle atoms), then the transposes
@@ -509,7 +542,7 @@ __global__ void __launch_bounds__(512, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1 + 4);  // the producer's expect-tx arrival + one per scale-stager warp
+      mbar_init(&full[s], kI8 ? 1 : 1 + 4);  // the producer's expect-tx arrival + one per scale-stager warp
       mbar_init(&empty[s], 1);
       mbar_init(&sf_landed[s], 1);
     }
@@ -555,21 +588,23 @@ __global__ void __launch_bounds__(512, 1)
               ok = false;
               break;
             }
-            const int ks = min(C::KSTEPS, args.k_steps - kb * C::KSTEPS);
-            const uint32_t sf_bytes = static_cast<uint32_t>(ks) * 512u;
             uint8_t* sa = ring + stage * C::STAGE_BYTES;
             uint8_t* sb = sa + C::A_BYTES;
-            uint8_t* ssfa = sb + C::B_BYTES;
-            uint8_t* ssfb = ssfa + C::SFA_BYTES;
-            mbar_arrive_expect_tx(&sf_landed[stage], sf_bytes * (1 + BN / 128));
-            bulk_load(ssfa, args.sfa + (static_cast<int64_t>(mb) * args.k_atoms + kb * C::KSTEPS) * 512, sf_bytes,
-                      &sf_landed[stage]);
+            if constexpr (!kI8) {
+              const int ks = min(C::KSTEPS, args.k_steps - kb * C::KSTEPS);
+              const uint32_t sf_bytes = static_cast<uint32_t>(ks) * 512u;
+              uint8_t* ssfa = sb + C::B_BYTES;
+              uint8_t* ssfb = ssfa + C::SFA_BYTES;
+              mbar_arrive_expect_tx(&sf_landed[stage], sf_bytes * (1 + BN / 128));
+              bulk_load(ssfa, args.sfa + (static_cast<int64_t>(mb) * args.k_atoms + kb * C::KSTEPS) * 512, sf_bytes,
+                        &sf_landed[stage]);
 #pragma unroll
-            for (int j = 0; j < BN / 128; ++j)
-              bulk_load(ssfb + j * C::KSTEPS * C::SF_ATOM_BYTES,
-                        args.sfb + (static_cast<int64_t>(b_row0<BN, KIND>(args, nb, j) / 128) * args.k_atoms +
-                                    kb * C::KSTEPS) * 512,
-                        sf_bytes, &sf_landed[stage]);
+              for (int j = 0; j < BN / 128; ++j)
+                bulk_load(ssfb + j * C::KSTEPS * C::SF_ATOM_BYTES,
+                          args.sfb + (static_cast<int64_t>(b_row0<BN, KIND>(args, nb, j) / 128) * args.k_atoms +
+                                      kb * C::KSTEPS) * 512,
+                          sf_bytes, &sf_landed[stage]);
+            }
             mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES);
             tma_load_2d(sa, &tmap_a, &full[stage], kb * C::BK_BYTES, mb * C::BM);
 #pragma unroll
@@ -590,7 +625,7 @@ __global__ void __launch_bounds__(512, 1)
         // its time limit instead)
         for (int s = 0; s < C::STAGES; ++s)
           if (armed_mask & (1u << s)) {
-            mbar_wait(&sf_landed[s], (armed_parity >> s) & 1u, never_abort, args.timeout_ns);
+            if (!kI8) mbar_wait(&sf_landed[s], (armed_parity >> s) & 1u, never_abort, args.timeout_ns);
             mbar_wait(&full[s], (armed_parity >> s) & 1u, never_abort, args.timeout_ns);
           }
       }
@@ -631,14 +666,22 @@ __global__ void __launch_bounds__(512, 1)
             const uint32_t sfb_t = sfa_t + C::SFA_COLS;
             if (kb * C::KSTEPS + C::KSTEPS <= args.k_steps) {
 #pragma unroll
-              for (int k = 0; k < C::KSTEPS; ++k)
-                tc_mma_nvf4(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::IDESC, accumulate | k, sfa_t + k * 4,
-                            sfb_t + k * (BN / 32));
+              for (int k = 0; k < C::KSTEPS; ++k) {
+                if constexpr (kI8)
+                  tc_mma_i8(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::IDESC, accumulate | k);
+                else
+                  tc_mma_nvf4(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::IDESC, accumulate | k, sfa_t + k * 4,
+                              sfb_t + k * (BN / 32));
+              }
             } else {
               const int ks = args.k_steps - kb * C::KSTEPS;  // K tail: 1 .. KSTEPS-1 steps
-              for (int k = 0; k < ks; ++k)
-                tc_mma_nvf4(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::IDESC, accumulate | k, sfa_t + k * 4,
-                            sfb_t + k * (BN / 32));
+              for (int k = 0; k < ks; ++k) {
+                if constexpr (kI8)
+                  tc_mma_i8(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::IDESC, accumulate | k);
+                else
+                  tc_mma_nvf4(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::IDESC, accumulate | k, sfa_t + k * 4,
+                              sfb_t + k * (BN / 32));
+              }
             }
             accumulate = 1;
             tc_commit(&empty[stage]);
@@ -668,65 +711,67 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp < 8) {
     regs_decrease<64>();
-    // ------------------------------------------------------------------ scale stagers
-    // Lane i of warp 4+q writes TMEM lane 32q+i.  The MMA reads, for row r of a 128-row block, the
-    // 4 scales of one K step from column r / 32 of that step's group of 4 columns, identically in
-    // every sub-partition; 16-byte row i of a 512-byte scale atom is exactly those 4 columns of lane i.
-    const int q = warp & 3;
-    constexpr int NV = C::SF_COLS / 4;  // 16-byte vectors per lane and stage
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int u = blockIdx.x; u < args.num_units; u += gridDim.x) {
-      const WorkUnit wu = work_unit(args, u, num_kb);
-      bool ok = true;
-      for (int kb = wu.kb0; kb < wu.kb1; ++kb) {
-        const bool got = mbar_wait(&sf_landed[stage], phase, abort_flag, args.timeout_ns);
-        if (!__all_sync(0xFFFFFFFFu, got)) {
-          ok = false;
+    if constexpr (!kI8) {  // the INT8 form has no block scales to stage
+      // ------------------------------------------------------------------ scale stagers
+      // Lane i of warp 4+q writes TMEM lane 32q+i.  The MMA reads, for row r of a 128-row block, the
+      // 4 scales of one K step from column r / 32 of that step's group of 4 columns, identically in
+      // every sub-partition; 16-byte row i of a 512-byte scale atom is exactly those 4 columns of lane i.
+      const int q = warp & 3;
+      constexpr int NV = C::SF_COLS / 4;  // 16-byte vectors per lane and stage
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int u = blockIdx.x; u < args.num_units; u += gridDim.x) {
+        const WorkUnit wu = work_unit(args, u, num_kb);
+        bool ok = true;
+        for (int kb = wu.kb0; kb < wu.kb1; ++kb) {
+          const bool got = mbar_wait(&sf_landed[stage], phase, abort_flag, args.timeout_ns);
+          if (!__all_sync(0xFFFFFFFFu, got)) {
+            ok = false;
+            break;
+          }
+          const uint8_t* ssfa = ring + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
+          const uint8_t* ssfb = ssfa + C::SFA_BYTES;
+          const int ks = min(C::KSTEPS, args.k_steps - kb * C::KSTEPS);
+          const uint32_t t_sf = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + C::SF_COL0 + stage * C::SF_COLS;
+          // slot column order: A steps 0..KSTEPS-1 (4 columns each), then for each step k the weight's
+          // 128-row blocks j = 0 .. BN/128-1 (4 columns each)
+  #pragma unroll
+          for (int grp = 0; grp < NV / 2; ++grp) {
+            uint32_t v[8];
+  #pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int idx = grp * 2 + h;
+              int k;
+              const uint8_t* src;
+              if (idx < C::KSTEPS) {
+                k = idx;
+                src = ssfa + k * C::SF_ATOM_BYTES;
+              } else {
+                k = (idx - C::KSTEPS) / (BN / 128);
+                src = ssfb + ((idx - C::KSTEPS) % (BN / 128)) * C::KSTEPS * C::SF_ATOM_BYTES + k * C::SF_ATOM_BYTES;
+              }
+              uint4 x = make_uint4(0, 0, 0, 0);
+              if (k < ks) x = *reinterpret_cast<const uint4*>(src + lane * 16);
+              v[4 * h + 0] = x.x;
+              v[4 * h + 1] = x.y;
+              v[4 * h + 2] = x.z;
+              v[4 * h + 3] = x.w;
+            }
+            tmem_st_32x32b_x8(t_sf + grp * 8, v);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) {
+          if (lane == 0) raise_device_error(args.error_word, kErrTimeout, abort_flag);
           break;
         }
-        const uint8_t* ssfa = ring + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
-        const uint8_t* ssfb = ssfa + C::SFA_BYTES;
-        const int ks = min(C::KSTEPS, args.k_steps - kb * C::KSTEPS);
-        const uint32_t t_sf = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + C::SF_COL0 + stage * C::SF_COLS;
-        // slot column order: A steps 0..KSTEPS-1 (4 columns each), then for each step k the weight's
-        // 128-row blocks j = 0 .. BN/128-1 (4 columns each)
-#pragma unroll
-        for (int grp = 0; grp < NV / 2; ++grp) {
-          uint32_t v[8];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int idx = grp * 2 + h;
-            int k;
-            const uint8_t* src;
-            if (idx < C::KSTEPS) {
-              k = idx;
-              src = ssfa + k * C::SF_ATOM_BYTES;
-            } else {
-              k = (idx - C::KSTEPS) / (BN / 128);
-              src = ssfb + ((idx - C::KSTEPS) % (BN / 128)) * C::KSTEPS * C::SF_ATOM_BYTES + k * C::SF_ATOM_BYTES;
-            }
-            uint4 x = make_uint4(0, 0, 0, 0);
-            if (k < ks) x = *reinterpret_cast<const uint4*>(src + lane * 16);
-            v[4 * h + 0] = x.x;
-            v[4 * h + 1] = x.y;
-            v[4 * h + 2] = x.z;
-            v[4 * h + 3] = x.w;
-          }
-          tmem_st_32x32b_x8(t_sf + grp * 8, v);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[stage]);
-        if (++stage == C::STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-      if (!ok) {
-        if (lane == 0) raise_device_error(args.error_word, kErrTimeout, abort_flag);
-        break;
       }
     }
   } else {
@@ -735,7 +780,7 @@ __global__ void __launch_bounds__(512, 1)
     const int e = (warp - 8) >> 2;
     const int q = warp & 3;
     uint8_t* xpose = xpose_all + (warp - 8) * C::XPOSE_BYTES;
-    const float alpha = __fmul_rn(*args.ga, *args.gb);
+    const float alpha_t = kI8 ? 1.0f : __fmul_rn(*args.ga, *args.gb);
     const float qg = args.q_codes != nullptr ? *args.q_g : 1.0f;
     int abuf = 0;
     uint32_t aphase = 0;
@@ -765,6 +810,13 @@ __global__ void __launch_bounds__(512, 1)
       if (++abuf == C::ACC_BUFS) {
         abuf = 0;
         aphase ^= 1u;
+      }
+      // the dequantisation factor of this row: ga * gb, or the INT8 form's activation scale of the row
+      // (0 for the padding rows past M, whose outputs the store drops)
+      float alpha = alpha_t;
+      if constexpr (kI8) {
+        alpha = row0 + lane < args.M ? __ldg(args.row_scale + row0 + lane) : 0.0f;
+        i8_scale_columns<BN, KIND>(args, e, nb, acc);
       }
       // (the head norm's sum of squares is taken while loading, so the host never splits QK-norm GEMMs)
       if (KIND != kEpiQkNorm && args.splits > 1 &&

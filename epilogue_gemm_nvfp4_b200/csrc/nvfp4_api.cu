@@ -28,6 +28,7 @@ struct DeviceState {
   int sm_count = 0;
   unsigned int* error_word = nullptr;
   bool smem_attr_set[2][4] = {};
+  bool smem_attr_set_i8[2][4] = {};  // the INT8 form of the one-CTA kernel
   int pair_clusters[2][4] = {};  // resident CTA pairs per (split-K, epilogue kind), 0 until first use
 };
 
@@ -517,3 +518,6 @@ nvfp4_status nvfp4_get_device_error(nvfp4_stream_t stream) {
 // Entry points of the bandwidth-bound op family (amax, quantise, fake quantise, adaLN quantise,
 // dequantise): they use the helpers above, so they are part of this translation unit.
 #include "quantize_api.cuh"
+
+// Entry points of the W8A8 INT8 linear and its quantiser.
+#include "int8_api.cuh"

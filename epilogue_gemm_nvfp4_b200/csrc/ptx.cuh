@@ -185,6 +185,17 @@ __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uin
       : "memory");
 }
 
+// D (s32, TMEM) (+)= A * B^T for signed 8-bit A and B, K = 32 per instruction (32 bytes of each row).
+__device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Paired (cta_group::2) forms: one warp of each CTA allocates / frees; the leader's single thread
 // issues MMAs for both CTAs and commits to the barriers of the CTAs in `cta_mask`.
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_slot, uint32_t ncols) {
@@ -312,6 +323,15 @@ __host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
          | (1u << 10)                                // B format: E2M1
          | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
          | (0u << 23)                                // scale format: UE4M3
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// Instruction descriptor of tcgen05.mma.kind::i8: s32 accumulator, signed 8-bit A and B, both K-major.
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
+  return (2u << 4)                                   // D format: S32
+         | (1u << 7)                                 // A format: signed 8-bit
+         | (1u << 10)                                // B format: signed 8-bit
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 

@@ -247,6 +247,47 @@ NVFP4_API nvfp4_status nvfp4_adaln_quantize(const void* x, int64_t rows, int64_t
                                             const nvfp4_adaln_desc* ada, int32_t compute_scale,
                                             const nvfp4_tensor* out, nvfp4_stream_t stream);
 
+/*
+ * W8A8 INT8 operands ("Quantizing a Dual-Branch Flow-Matching Diffusion Transformer for Consumer GPUs",
+ * method section: per-output-row INT8 weights, per-token dynamic INT8 activations, SmoothQuant channel
+ * migration).  A `rows` x `cols` tensor:
+ *   q:      int8 [rows, ld] (row stride ld bytes; 0 means cols), values in [-127, 127];
+ *   scale:  fp32 [rows], the decode scale of each row: value = q * scale[row].
+ */
+typedef struct {
+  void* q;
+  float* scale;
+  int64_t rows;
+  int64_t cols;
+  int64_t ld;
+} nvfp4_int8_tensor;
+
+/*
+ * Quantise bf16 x [rows, cols] (row stride ldx elements) to per-row INT8 into `out` (out->rows == rows,
+ * out->cols == cols).  For each row, each step one binary32 operation rounded to nearest even:
+ *   x'[k] = x[k] * col_mult[k]   (col_mult = NULL: x' = x)
+ *   s     = max_k |x'| / 127     (1 for an all-zero row), stored in out->scale[row]
+ *   q[k]  = clamp(RNE(x'[k] * (127 / max_k |x'|)), -127, 127)   (0 for an all-zero row)
+ * col_mult carries the SmoothQuant migration: 1 / lambda for activations, lambda for the weight (whose
+ * rows are the output channels).  Rules: cols % 16 == 0; x, ldx * 2, col_mult, out->q and out->ld 16-byte
+ * aligned; out->scale 4-byte aligned.
+ */
+NVFP4_API nvfp4_status nvfp4_int8_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx,
+                                           const float* col_mult, const nvfp4_int8_tensor* out,
+                                           nvfp4_stream_t stream);
+
+/*
+ * The fused W8A8 linear: out = epilogue(y) with y[m,n] = (sum_k a.q[m,k] * w.q[n,k]) * a.scale[m] *
+ * w.scale[n], the products summed exactly in s32 on the tensor cores (tcgen05.mma.kind::i8), then
+ * converted to fp32 and scaled.  `epi`, out_bf16, ld_out and out_fp4 mean what they mean for
+ * nvfp4_linear, every epilogue kind included.  Rules: K % 32 == 0; N % 128 == 0 (N % 256 == 0 for QKNORM
+ * and GATED_SILU); a.q, w.q and their ld 16-byte aligned; a.scale and w.scale 16-byte aligned.  There
+ * is no split of K: the s32 sums of K <= 131072 cannot overflow.
+ */
+NVFP4_API nvfp4_status nvfp4_int8_linear(const nvfp4_int8_tensor* a, const nvfp4_int8_tensor* w,
+                                         const nvfp4_epilogue_desc* epi, void* out_bf16, int64_t ld_out,
+                                         const nvfp4_tensor* out_fp4, nvfp4_stream_t stream);
+
 /* Dequantise t to bf16 [t->rows, ld_out]: value = e2m1(code) * (e4m3(scale) * g), each product in fp32
  * rounded to nearest even, then rounded to bf16.  Rules as for nvfp4_quantize. */
 NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor* t, void* out_bf16, int64_t ld_out, nvfp4_stream_t stream);

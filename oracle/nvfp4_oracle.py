@@ -385,19 +385,22 @@ def smoothquant_factors(act_absmax, w, alpha: float = 0.5):
     return lam.astype(F32)
 
 
-def int8_quantize_rows(x, smooth=None):
+def int8_quantize_rows(x, act_mult=None):
     """Symmetric per-row INT8 ([Dual-Branch], method: per-token dynamic activations and per-output-row
     weights).  Each step is one binary32 operation rounded to nearest even:
-        x'  = x / smooth[k]         (when a smoothing vector is given)
-        s   = max_k |x'| / 127      (1 for an all-zero row)
-        q   = clamp(RNE(x' / s), -127, 127)
+        x'  = x * act_mult[k]        (the SmoothQuant divide, as a multiply by act_mult = 1 / lambda)
+        s   = max_k |x'| / 127       (the decode scale; 1 for an all-zero row)
+        inv = 127 / max_k |x'|       (0 for an all-zero row)
+        q   = clamp(RNE(x' * inv), -127, 127)
     x float32 [M, K] -> (q int8 [M, K], s float32 [M])."""
     x = np.asarray(x, dtype=F32)
-    if smooth is not None:
-        x = (x / np.asarray(smooth, dtype=F32)[None, :]).astype(F32)
+    if act_mult is not None:
+        x = (x * np.asarray(act_mult, dtype=F32)[None, :]).astype(F32)
     amax = np.max(np.abs(x), axis=1).astype(F32) if x.shape[1] else np.zeros(x.shape[0], F32)
-    s = np.where(amax == 0, F32(1.0), (amax / F32(127.0)).astype(F32)).astype(F32)
-    v = (x / s[:, None]).astype(F32)
+    zero = amax == 0
+    s = np.where(zero, F32(1.0), (amax / F32(127.0)).astype(F32)).astype(F32)
+    inv = np.where(zero, F32(0.0), (F32(127.0) / np.where(zero, F32(1.0), amax)).astype(F32)).astype(F32)
+    v = (x * inv[:, None]).astype(F32)
     q = np.clip(np.rint(v), -127, 127).astype(np.int8)      # rint: ties to even
     return q, s
 

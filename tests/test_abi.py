@@ -125,6 +125,26 @@ def test_argument_checks_return_before_any_launch(lib):
     assert ada(rstd=0x10002) == B.ERR_MISALIGNED
     assert ada(u_out=0x10008) == B.ERR_MISALIGNED
     assert ada(ld_u=516) == B.ERR_MISALIGNED
+    # W8A8 INT8
+    i8 = lambda rows, cols, ptr=0x10000, ld=0, scale=0x10000: B.CInt8Tensor(ptr, scale, rows, cols, ld)
+    iq = lambda x=0x10000, rows=4, cols=512, ldx=512, mult=None, t=None: lib.nvfp4_int8_quantize(
+        x, rows, cols, ldx, mult, ctypes.byref(t if t is not None else i8(rows, cols)), None)
+    assert iq(x=None) == B.ERR_INVALID_ARG
+    assert iq(t=i8(5, 512)) == B.ERR_INVALID_ARG                                         # rows differ
+    assert iq(cols=520, ldx=520, t=i8(4, 520, ld=528)) == B.ERR_UNSUPPORTED_SHAPE
+    assert iq(ldx=516) == B.ERR_MISALIGNED
+    assert iq(mult=0x10004) == B.ERR_MISALIGNED
+    assert iq(t=i8(4, 512, ld=520)) == B.ERR_MISALIGNED                                   # ld % 16
+    assert iq(t=i8(4, 512, scale=0x10002)) == B.ERR_MISALIGNED
+    assert lib.nvfp4_int8_quantize(0x10000, 4, 512, 512, None, None, None) == B.ERR_INVALID_ARG
+    il = lambda a_, w_, d_=desc, out=0x10000, ld=512: lib.nvfp4_int8_linear(
+        ctypes.byref(a_), ctypes.byref(w_), ctypes.byref(d_), out, ld, None, None)
+    assert il(i8(256, 512), i8(512, 256)) == B.ERR_INVALID_ARG                            # K mismatch
+    assert il(i8(256, 48), i8(512, 48)) == B.ERR_UNSUPPORTED_SHAPE                        # K % 32
+    assert il(i8(256, 512), i8(200, 512)) == B.ERR_UNSUPPORTED_SHAPE                      # N % 128
+    assert il(i8(256, 512, scale=0x10004), i8(512, 512)) == B.ERR_MISALIGNED              # scales 16-byte aligned
+    assert il(i8(256, 512), i8(512, 512), out=0x10002) == B.ERR_MISALIGNED
+    assert il(i8(256, 512), i8(512, 512), d_=B.CEpilogue(kind=9)) == B.ERR_INVALID_ARG
 
 
 @pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-device path")
@@ -132,6 +152,9 @@ def test_valid_call_without_a_device_reports_cuda_error(lib):
     a, w = _tensor(256, 512), _tensor(512, 512)
     desc = B.CEpilogue()
     assert lib.nvfp4_linear(ctypes.byref(a), ctypes.byref(w), ctypes.byref(desc), 0x10000, 512, None, None) \
+        == B.ERR_CUDA
+    a8, w8 = B.CInt8Tensor(0x10000, 0x10000, 256, 512, 0), B.CInt8Tensor(0x10000, 0x10000, 512, 512, 0)
+    assert lib.nvfp4_int8_linear(ctypes.byref(a8), ctypes.byref(w8), ctypes.byref(desc), 0x10000, 512, None, None) \
         == B.ERR_CUDA
 
 
@@ -141,7 +164,8 @@ def test_ctypes_structs_match_the_header(tmp_path):
     import subprocess
     if shutil.which("gcc") is None:
         pytest.skip("gcc not available")
-    structs = {"nvfp4_tensor": B.CTensor, "nvfp4_epilogue_desc": B.CEpilogue, "nvfp4_adaln_desc": B.CAdaln}
+    structs = {"nvfp4_tensor": B.CTensor, "nvfp4_epilogue_desc": B.CEpilogue, "nvfp4_adaln_desc": B.CAdaln,
+               "nvfp4_int8_tensor": B.CInt8Tensor}
     lines = ['#include <stdio.h>', '#include "nvfp4.h"', "int main(void) {"]
     for cname, py in structs.items():
         lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')

@@ -499,7 +499,7 @@ def test_int8_rows_ties_extremes_and_zero_rows():
     assert q[0].tolist() == [127, 0, 2, 2, -2, 0, 126, -3]
     assert q[1].tolist() == [0] * 8
     assert q[2, 0] == -127 and s[2] == np.float32(4.0) / np.float32(127.0)
-    assert q[2, 1] == 32                                         # 1 / (4/127) = 31.75 -> 32
+    assert q[2, 1] == 32                                         # 1 * 127/4 = 31.75 -> 32
 
 
 def test_int8_rows_within_half_a_step_of_the_exact_quotient():
@@ -519,9 +519,9 @@ def test_int8_rows_within_half_a_step_of_the_exact_quotient():
 def test_int8_smoothing_divides_each_input_channel():
     rng = np.random.default_rng(10)
     x = rng.standard_normal((4, 32)).astype(np.float32)
-    lam = np.ones(32, np.float32)
-    lam[5] = 4.0
-    q1, s1 = O.int8_quantize_rows(x, lam)
+    mult = np.ones(32, np.float32)
+    mult[5] = 0.25                                               # lambda = 4 for channel 5
+    q1, s1 = O.int8_quantize_rows(x, mult)
     x2 = x.copy()
     x2[:, 5] /= 4.0
     q2, s2 = O.int8_quantize_rows(x2)
