@@ -39,6 +39,26 @@ def normwise_rel_err(got, ref) -> float:
     return O.rel_err_normwise(got, ref)
 
 
+def assert_close(got, ref, what, tol=2e-2):
+    """The parity bar of a GEMM + epilogue output (bf16) against the oracle's fp64 value: the normwise max
+    relative error max|got - ref| / max|ref| <= tol, and element by element |got - ref| <= tol *
+    max(|ref|, 1e-2 * rms(ref)), so that a wrong bias, a misplaced column block or a wrong small value
+    fails even where the largest outputs hide it from the normwise measure.  Returns the normwise error."""
+    got = np.asarray(got)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = normwise_rel_err(got, ref)
+    assert err <= tol, f"{what}: normwise rel err {err:.3e} > {tol}"
+    worst = elementwise_ok(got, ref, rel=tol)
+    if worst > 1.0:
+        ref64 = np.asarray(ref, np.float64)
+        rms = np.sqrt(np.mean(ref64 * ref64))
+        ratio = np.abs(np.asarray(got, np.float64) - ref64) / np.maximum(np.abs(ref64), 1e-2 * rms)
+        idx = np.unravel_index(np.argmax(ratio), ratio.shape)
+        raise AssertionError(f"{what}: elementwise error {worst * tol:.3e} relative at {idx}: got {got[idx]}, "
+                             f"oracle {ref64[idx]}")
+    return err
+
+
 def elementwise_ok(got, ref, rel=2e-2, floor_frac=1e-2):
     """Elementwise |got-ref| <= rel * max(|ref|, floor_frac * rms(ref)); returns the worst ratio."""
     ref = np.asarray(ref, np.float64)
