@@ -171,15 +171,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&p);
 }
 
-// silu(a) = a * sigmoid(a) = h + h * tanh(h) with h = a / 2: one hardware tanh (tanh.approx.f32,
-// relative error about 2^-11, far below the bf16 output's 2^-8) instead of an exponential and a
-// reciprocal.
-__device__ __forceinline__ float silu(float a) {
-  const float h = 0.5f * a;
-  float t;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
-  return fmaf(h, t, h);
-}
+// silu(a) = a / (1 + exp(-a)), with the fast exponential and division intrinsics: a few fp32 ulps of
+// relative error for every a.  (The form h + h * tanh(h), h = a / 2, cancels for negative a: there
+// tanh is near -1, and the hardware tanh's 2^-11 relative error became several percent of silu(a)
+// at a = -5.)  For a below about -88 the exponential overflows and the quotient is -0.
+__device__ __forceinline__ float silu(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 
 __device__ __forceinline__ void tmem_load32(uint32_t taddr, float* v) {
   uint32_t r[32];
@@ -301,7 +297,9 @@ __device__ __forceinline__ void emit_row32(const GemmArgs& a, const OutMaps* om,
     xpose_acquire();
     *reinterpret_cast<uint4*>(xpose + lane * 16) = make_uint4(words[0], words[1], words[2], words[3]);
     xpose_release(&om->q_codes, xpose, col0 / 2, row0, a.M);
-    if (row < a.num_m_blocks * 128)  // the scale layout's rows end at the 128-row padding
+    // the scale layout's rows end at the 128-row padding and its blocks at the 4-block padding of a row
+    // (a ragged N's last tile reaches past both; its blocks up to the padding get zero scales)
+    if (row < a.num_m_blocks * 128 && col0 / 16 < 4 * a.q_k_atoms)
       *reinterpret_cast<uint16_t*>(a.q_scales + scale_offset(row, col0 / 16, a.q_k_atoms)) =
           static_cast<uint16_t>(sc[0] | (sc[1] << 8));
   }
@@ -400,10 +398,20 @@ struct Epilogue {
         float* y = acc + 32 * c;
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
+          // N is a multiple of 16, so a 16-column group lies wholly inside or wholly past it; the last
+          // 128-wide tile of a ragged N reads no bias, residual or gate past N (its accumulator columns
+          // there are 0: the weight's TMA box fills the rows past N with zeros) and the store map drops
+          // those columns
+          const bool in_n = col0 + 16 * g < a.N;
           float b[16];
-          if (a.bias != nullptr) load_bf16x16(a.bias + col0 + 16 * g, b);
+          if (a.bias != nullptr && in_n) {
+            load_bf16x16(a.bias + col0 + 16 * g, b);
+          } else {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) y[16 * g + i] = y[16 * g + i] * alpha + (a.bias != nullptr ? b[i] : 0.0f);
+            for (int i = 0; i < 16; ++i) b[i] = 0.0f;
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) y[16 * g + i] = y[16 * g + i] * alpha + b[i];
           if (KIND == kEpiQkNorm && gamma != nullptr) {
             float gm[16];
             load_bf16x16(gamma + COLS * e + 32 * c + 16 * g, gm);
@@ -412,7 +420,7 @@ struct Epilogue {
           }
           if constexpr (KIND == kEpiResidGate) {
             float r[16];
-            if (row < a.M) {
+            if (row < a.M && in_n) {
               load_bf16x16(a.residual + static_cast<int64_t>(row) * a.ld_res + col0 + 16 * g, r);
             } else {
 #pragma unroll
@@ -421,7 +429,7 @@ struct Epilogue {
             const float4* gp = reinterpret_cast<const float4*>(a.gate + col0 + 16 * g);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
-              const float4 gg = __ldg(gp + v);
+              const float4 gg = in_n ? __ldg(gp + v) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
               y[16 * g + 4 * v + 0] = fmaf(gg.x, y[16 * g + 4 * v + 0], r[4 * v + 0]);
               y[16 * g + 4 * v + 1] = fmaf(gg.y, y[16 * g + 4 * v + 1], r[4 * v + 1]);
               y[16 * g + 4 * v + 2] = fmaf(gg.z, y[16 * g + 4 * v + 2], r[4 * v + 2]);
