@@ -41,11 +41,15 @@ NOMINAL_FP4_TFLOPS = 9000.0   # NVIDIA's dense FP4 figure for B200
 BF16_TO_FP4 = 4.0             # nominal dense FP4 / dense bf16 tensor-core rate (9 / 2.25)
 
 
-TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "nvfp4_gemm_up_dram_2048sq.md")
+#: the DRAM traffic of one full-size launch of the dominant kernel, written with its ncu capture
+TRAFFIC_DATA = os.path.join(ROOT, "profiles", "nvfp4_gemm_up_dram_2048sq.json")
 
 
 #: the sources the up-projection GEMM is built from: its device code and the host code that launches it
 GEMM_SOURCES = ("ptx.cuh", "quantize.cuh", "gemm.cuh", "gemm_pair.cuh", "nvfp4_api.cu")
+
+#: FP4 tensor-core rate of one SM: a 128 x 256 x 64 block-scaled MMA every 128 cycles
+FP4_FLOP_PER_CLK_SM = 32768
 
 
 def _code_only(text: str) -> str:
@@ -71,18 +75,14 @@ def library_sources_sha256():
 
 
 def measured_traffic():
-    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, or None when the
+    """DRAM bytes per launch of the dominant kernel from the committed capture record, or None when the
     library's sources have changed since those counters were taken."""
     try:
-        fields = {}
-        with open(TRAFFIC_PROFILE) as fh:
-            for line in fh:
-                if ":" in line:
-                    k, v = line.split(":", 1)
-                    fields[k.strip()] = v.strip()
-        if fields.get("sources_sha256") != library_sources_sha256():
+        with open(TRAFFIC_DATA) as fh:
+            rec = json.load(fh)
+        if rec.get("sources_sha256") != library_sources_sha256():
             return None
-        return int(fields["traffic_bytes_per_launch"])
+        return int(rec["traffic_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
         return None
 
@@ -398,7 +398,13 @@ def run_native(args, ws, rank, local):
     pk = peaks()
     dominant = max(("qkv", "out", "up", "down"), key=lambda k: fl[k])
     achieved = fl[dominant] / (per_op[dominant] * 1e-3) / 1e12
-    peak_fp4 = pk["bf16_sus"] * BF16_TO_FP4
+    clocks = clk.summary()
+    # the burst bf16 figure for a region under a second (the clock stays near its maximum there), the
+    # sustained one for a region long enough to settle under the power cap
+    sustained = ms > 1000.0
+    peak_fp4 = (pk["bf16_sus"] if sustained else pk["bf16"]) * BF16_TO_FP4
+    sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    at_clock = (FP4_FLOP_PER_CLK_SM * sm_count * clocks["sm_mhz"] * 1e6 / 1e12) if clocks.get("sm_mhz") else None
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
@@ -410,14 +416,20 @@ def run_native(args, ws, rank, local):
         "frac_of_nominal_fp4": round(value / ws / NOMINAL_FP4_TFLOPS, 4),
         "per_op_us": {k: round(v * 1e3, 1) for k, v in per_op.items()},
         "per_gemm_tflops": {k: round(fl[k] / (per_op[k] * 1e-3) / 1e12, 1) for k in ("qkv", "out", "up", "down")},
-        "roofline": {"bound": "tensor", "kernel": f"nvfp4_gemm_kernel ({dominant}: gated SiLU + requant)",
+        "roofline": {"bound": "tensor",
+                     "kernel": f"nvfp4_gemm_pair_kernel ({dominant}: gated SiLU + NVFP4 requant, CTA pairs)",
                      "achieved": round(achieved, 1), "peak": round(peak_fp4, 1), "unit": "TFLOP/s",
                      "frac": round(achieved / peak_fp4, 4),
-                     "peak_note": f"{pk['src']} sustained bf16 {pk['bf16_sus']} x {BF16_TO_FP4} (nominal FP4/bf16)",
+                     "peak_note": (f"{pk['src']} {'sustained' if sustained else 'burst'} bf16 "
+                                   f"{pk['bf16_sus'] if sustained else pk['bf16']} x {BF16_TO_FP4} (nominal FP4/bf16 "
+                                   f"ratio); the timed region ran {ms:.0f} ms"),
                      "frac_of_nominal_9pf": round(achieved / NOMINAL_FP4_TFLOPS, 4),
+                     "peak_at_sampled_clock": round(at_clock, 1) if at_clock else None,
+                     "frac_at_sampled_clock": round(achieved / at_clock, 4) if at_clock else None,
+                     "at_clock_note": f"{FP4_FLOP_PER_CLK_SM} FLOP/clock/SM x {sm_count} SMs x the median sampled SM clock",
                      "traffic": measured_traffic(),
-                     "traffic_note": "bytes per launch, ncu dram read+write of the full-size launch "
-                                     "(profiles/nvfp4_gemm_up_dram_2048sq.md); null once the kernel sources change"},
+                     "traffic_note": "bytes per launch, ncu dram read+write of one full-size launch "
+                                     "(profiles/nvfp4_gemm_up_dram_2048sq.json); null once the kernel sources change"},
         "quantize_roofline": None,
         "e2e": {"value": round(step_flops * ws / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -436,7 +448,7 @@ def run_native(args, ws, rank, local):
                                         "the whole dynamic-scale op; achieved_two_pass also counts the amax pass's "
                                         "2 B/elem read, which the dynamic scale needs because every element's code "
                                         "depends on the tensor amax and the 156 MB tensor exceeds L2"}
-    out["clocks"] = clk.summary()
+    out["clocks"] = clocks
     if rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
     return out
