@@ -85,9 +85,10 @@ nvfp4_status nvfp4_int8_linear(const nvfp4_int8_tensor* a, const nvfp4_int8_tens
   if (w->cols != K) return NVFP4_ERR_INVALID_ARG;
   if (epi->kind < NVFP4_EPI_BIAS || epi->kind > NVFP4_EPI_RESID_GATE) return NVFP4_ERR_INVALID_ARG;
   if (K % 32 || K > 131072) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  // tile width as in the FP4 linear (the FP4 rule on K is in elements of 64; here K counts bytes)
+  // tile width as in the FP4 linear (the FP4 rule on K is in elements of 64; here K counts bytes); the
+  // INT8 epilogue reads a weight scale for every column of a tile, so N stays a multiple of 128
   const int BN = tile_n_for(N, 64, epi->kind);
-  if (BN == 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (BN == 0 || N % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(a->scale) || !aligned16(w->scale)) return NVFP4_ERR_MISALIGNED;
   const int64_t n_out = epi->kind == NVFP4_EPI_GATED_SILU ? N / 2 : N;

@@ -233,12 +233,16 @@ nvfp4_status make_store_maps(OutMaps* om, void* out_bf16, int64_t ld_out, const 
 // its sum of squares while loading the accumulator and is never split.
 int split_k_for(int64_t K, int32_t kind) { return (K >= 32768 && kind != NVFP4_EPI_QKNORM) ? 2 : 1; }
 
+// Column tile width: 256 whenever N allows it (CTA pairs); otherwise 128-wide tiles on single CTAs, the
+// last of which is ragged when N is not a multiple of 128 (the weight's TMA box fills its rows past N
+// with zeros, the epilogue reads no bias, residual or gate there and the store map drops its columns).
+// The head norm needs whole 256-wide heads and the gated SiLU pairs 128-row halves of a and b.
 int tile_n_for(int64_t N, int64_t K, int32_t kind) {
-  if (K < 64 || K % 64) return 0;
-  if (kind == NVFP4_EPI_QKNORM || kind == NVFP4_EPI_GATED_SILU) return (N > 0 && N % 256 == 0) ? 256 : 0;
+  if (K < 64 || K % 64 || N <= 0) return 0;
+  if (kind == NVFP4_EPI_QKNORM || kind == NVFP4_EPI_GATED_SILU) return N % 256 == 0 ? 256 : 0;
   if (kind == NVFP4_EPI_BIAS || kind == NVFP4_EPI_RESID_GATE) {
-    if (N > 0 && N % 256 == 0) return 256;
-    if (N > 0 && N % 128 == 0) return 128;
+    if (N % 256 == 0) return 256;
+    if (N % 16 == 0) return 128;
   }
   return 0;
 }
@@ -404,7 +408,7 @@ nvfp4_status linear_impl(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvf
   g.N = static_cast<int32_t>(N);
   g.K = static_cast<int32_t>(K);
   g.num_m_blocks = static_cast<int32_t>((M + 127) / 128);
-  g.num_n_blocks = static_cast<int32_t>(epi->kind == NVFP4_EPI_GATED_SILU ? (N / 2) / 128 : N / BN);
+  g.num_n_blocks = static_cast<int32_t>(epi->kind == NVFP4_EPI_GATED_SILU ? (N / 2) / 128 : (N + BN - 1) / BN);
   g.num_tiles = g.num_m_blocks * g.num_n_blocks;
   g.num_m_pairs = static_cast<int32_t>((M + 255) / 256);
   g.k_steps = static_cast<int32_t>(K / 64);

@@ -129,6 +129,9 @@ typedef struct {
 /*
  * Quantise a bf16 matrix x [rows, cols] (row stride ldx elements) to NVFP4 into `out`
  * (out->rows == rows, out->cols == cols).
+ * Passage: "Serving sub-second Ideogram v4 without quality loss", the paragraph on the 6x speed-up and
+ * NVFP4: the DiT's products run on 4-bit floats that Blackwell's tensor cores take natively, so every
+ * activation entering a product is first put in that format (the encoding above is the reading of it).
  *   compute_scale = 1: compute g = amax(|x|) / 2688 (1 when x is all zeros or empty) on the device and
  *                      store it in *out->tensor_scale: two stream-ordered kernels, an amax pass whose
  *                      last CTA writes g, then the quantise pass.  The first such call on a stream
@@ -143,11 +146,18 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols,
 
 /*
  * The fused NVFP4 linear: out = epilogue(a x w^T) on one GPU.
+ * Passages: "Serving sub-second Ideogram v4 without quality loss", the paragraph on kernel fusion (the
+ * small ops that follow a product, RMSNorm over 256-wide attention heads that straddle two tile fragments
+ * and the gated SiLU, run inside the GEMM instead of after a round trip of its output through memory);
+ * "Faster Ideogram 4 with Less Prompt Compute", "Most of the Tensor Was Zero" (the 53248 -> 4608 text
+ * projection with a bias, and a linear treats its rows independently) and "The NF4 Exactness Problem"
+ * (a kernel chosen by row count changes the bits, so nothing here depends on M).
  *   a:        NVFP4 [M, K] activation.  w: NVFP4 [N, K] weight (nn.Linear layout).
  *   out_bf16: bf16 [M, ld_out] (row stride in elements) or NULL when only out_fp4 is wanted.
  *   out_fp4:  NVFP4 [M, n_out] when epi->out_nvfp4 == 1, else ignored (may be NULL).
- * Rules: K % 64 == 0, K >= 64; N % 128 == 0 (N % 256 == 0 for QKNORM and GATED_SILU); M >= 1 (any);
- * all pointers and ld_out * 2 16-byte aligned.  The per-row arithmetic does not depend on M: row m of
+ * Rules: K % 64 == 0, K >= 64; N % 16 == 0 (N % 256 == 0 for QKNORM and GATED_SILU); M >= 1 (any);
+ * all pointers and ld_out * 2 16-byte aligned; the scale padding of w (rows past N up to a multiple of
+ * 128) holds zeros, as nvfp4_quantize writes it.  The per-row arithmetic does not depend on M: row m of
  * the output is bitwise the same whatever rows accompany it.
  * Kernels: 256-wide tiles (N % 256 == 0) run on two-CTA clusters with the paired tensor-core MMA;
  * other tiles on single CTAs.  The environment variable NVFP4_GEMM_PAIR=0, read once per process,
@@ -289,7 +299,10 @@ NVFP4_API nvfp4_status nvfp4_int8_linear(const nvfp4_int8_tensor* a, const nvfp4
                                          const nvfp4_tensor* out_fp4, nvfp4_stream_t stream);
 
 /* Dequantise t to bf16 [t->rows, ld_out]: value = e2m1(code) * (e4m3(scale) * g), each product in fp32
- * rounded to nearest even, then rounded to bf16.  Rules as for nvfp4_quantize. */
+ * rounded to nearest even, then rounded to bf16.  Rules as for nvfp4_quantize.
+ * Passage: the decode of the 4-bit format of "Serving sub-second Ideogram v4 without quality loss"
+ * (paragraph on NVFP4), in the reading above: a value is its E2M1 element times its block's E4M3 scale
+ * times the tensor's fp32 scale. */
 NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor* t, void* out_bf16, int64_t ld_out, nvfp4_stream_t stream);
 
 /* max |x| over a bf16 matrix into *amax (device fp32), overwriting it.  The first pass of

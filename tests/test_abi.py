@@ -47,7 +47,10 @@ def test_tile_choice_depends_on_n_k_kind_only(lib):
     assert B.tile_n(384, 512, "bias") == 128
     assert B.tile_n(384, 512, "qknorm") == 0          # heads need 256-column tiles
     assert B.tile_n(512, 96, "bias") == 0             # K % 64
-    assert B.tile_n(200, 512, "bias") == 0            # N % 128
+    assert B.tile_n(200, 512, "bias") == 0            # N % 16
+    assert B.tile_n(400, 512, "bias") == 128          # ragged last tile
+    assert B.tile_n(4624, 4608, "resid_gate") == 128
+    assert B.tile_n(400, 512, "gated_silu") == 0      # a and b halves pair 128-row blocks
 
 
 def _tensor(rows, cols, ptr=0x10000):
@@ -62,7 +65,7 @@ def test_argument_checks_return_before_any_launch(lib):
     assert lib.nvfp4_linear(None, ctypes.byref(w), ctypes.byref(desc), 0x10000, 512, None, None) == B.ERR_INVALID_ARG
     assert lin(_tensor(256, 512), _tensor(512, 256), desc) == B.ERR_INVALID_ARG          # K mismatch
     assert lin(_tensor(256, 96), _tensor(512, 96), desc) == B.ERR_UNSUPPORTED_SHAPE      # K % 64
-    assert lin(_tensor(256, 512), _tensor(200, 512), desc) == B.ERR_UNSUPPORTED_SHAPE    # N % 128
+    assert lin(_tensor(256, 512), _tensor(200, 512), desc) == B.ERR_UNSUPPORTED_SHAPE    # N % 16
     assert lin(_tensor(256, 512, 0x10008), w, desc) == B.ERR_MISALIGNED
     assert lin(a, w, desc, out=0x10002) == B.ERR_MISALIGNED
     assert lin(a, w, desc, ld=100) == B.ERR_INVALID_ARG                                    # ld_out < N
@@ -217,6 +220,6 @@ int main(void) {
     assert int(out[0]) == O.scale_buffer_bytes(300, 208)
     assert int(out[1]) == O.scale_atom_offset(130, 5, 208)
     assert int(out[2]) == B.ERR_UNSUPPORTED_SHAPE          # cols % 16
-    assert int(out[3]) == B.ERR_UNSUPPORTED_SHAPE          # N % 128
+    assert int(out[3]) == B.ERR_UNSUPPORTED_SHAPE          # N % 16
     assert int(out[4]) == 256
     assert " ".join(out[5:]).startswith("misaligned")
