@@ -47,6 +47,7 @@ static_assert(kStageKSteps == 2 || kStageKSteps == 4, "stage depth");
 
 struct GemmArgs {
   int32_t M, N, K;
+  int32_t n_out;         // output columns: N, or N / 2 for the gated SiLU
   int32_t num_m_blocks, num_n_blocks, num_tiles;
   int32_t num_m_pairs;   // 256-row blocks (CTA-pair kernel)
   int32_t k_steps;      // K / 64
@@ -71,6 +72,9 @@ struct GemmArgs {
   const float* q_g;
   int32_t q_k_atoms;
   unsigned int* out_amax_bits;  // raised to max |bf16 output| (fp32 bit pattern), or nullptr
+  // tile order of the persistent walk: 0 = row blocks fastest (a wave shares few weight blocks and
+  // keeps A resident in L2), 1 = column blocks fastest (a wave shares few row blocks and keeps W resident)
+  int32_t n_fastest;
   const float* row_scale;       // INT8 form: decode scale of each row of A [M]
   const float* col_scale;       // INT8 form: decode scale of each row of W [N]
   unsigned int* error_word;
@@ -81,6 +85,11 @@ struct GemmArgs {
   int32_t num_units;     // num_tiles * splits
   float* split_partials; // [num_tiles][2][128][cols per thread] fp32
   unsigned int* split_flags;  // [num_tiles], zero before the launch
+#ifdef NVFP4_TEST_HOOKS
+  // test builds only: the first unit of each split tile parks its partial but never publishes it, so the
+  // second unit's bounded wait runs out and the call reports a device timeout
+  int32_t test_withhold_split_ready;
+#endif
 };
 
 struct WorkUnit {
@@ -91,8 +100,13 @@ __device__ __forceinline__ WorkUnit work_unit(const GemmArgs& a, int u, int num_
   WorkUnit w;
   const int split = u % a.splits;
   w.tile = u / a.splits;
-  w.mb = w.tile % a.num_m_blocks;
-  w.nb = w.tile / a.num_m_blocks;
+  if (a.n_fastest) {
+    w.nb = w.tile % a.num_n_blocks;
+    w.mb = w.tile / a.num_n_blocks;
+  } else {
+    w.mb = w.tile % a.num_m_blocks;
+    w.nb = w.tile / a.num_m_blocks;
+  }
   w.kb0 = split * num_kb / a.splits;
   w.kb1 = (split + 1) * num_kb / a.splits;
   return w;
@@ -204,12 +218,13 @@ __device__ __forceinline__ void xpose_acquire() {
   __syncwarp();
 }
 
-// Hand the warp's buffer to the TMA engine as the box at (x, y) of `map` (nothing to store when the
-// box starts at or past the last row).
-__device__ __forceinline__ void xpose_release(const CUtensorMap* map, const uint8_t* xpose, int x, int y, int rows) {
+// Hand the warp's buffer to the TMA engine as the box at (x, y) of `map`.  `live` is false when the box
+// starts at or past the last row or the last column of the output: nothing is stored then (a box that
+// starts inside the output and reaches past its edge is clipped by the engine).
+__device__ __forceinline__ void xpose_release(const CUtensorMap* map, const uint8_t* xpose, int x, int y, bool live) {
   fence_proxy_async_smem();  // this thread's shared-memory writes become visible to the TMA engine
   __syncwarp();
-  if ((threadIdx.x & 31) == 0 && y < rows) {
+  if ((threadIdx.x & 31) == 0 && live) {
     tma_store_2d(map, xpose, x, y);
     bulk_commit_group();
   }
@@ -218,7 +233,7 @@ __device__ __forceinline__ void xpose_release(const CUtensorMap* map, const uint
 // Store 16 bf16 values of this lane's row at column col0: lane i writes row i of the 32 x 32-byte box
 // in the 32-byte swizzle (the two 16-byte halves swap every 4 rows, which also keeps the shared-memory
 // writes free of bank conflicts), then the box goes out with one TMA store.
-__device__ __forceinline__ void store_row16_bf16(const OutMaps* om, uint8_t* xpose, int row0, int col0, int rows,
+__device__ __forceinline__ void store_row16_bf16(const OutMaps* om, uint8_t* xpose, int row0, int col0, bool live,
                                                  const uint32_t* w) {
   const int lane = threadIdx.x & 31;
   const int sw = (lane >> 2) & 1;
@@ -226,13 +241,13 @@ __device__ __forceinline__ void store_row16_bf16(const OutMaps* om, uint8_t* xpo
   uint4* mine = reinterpret_cast<uint4*>(xpose + lane * 32);
   mine[sw] = make_uint4(w[0], w[1], w[2], w[3]);
   mine[sw ^ 1] = make_uint4(w[4], w[5], w[6], w[7]);
-  xpose_release(&om->out, xpose, col0, row0, rows);
+  xpose_release(&om->out, xpose, col0, row0, live);
 }
 
 // Store 32 bf16 values of this lane's row at column col0 as one 32-row x 64-byte box in the 64-byte
 // swizzle (16-byte chunk j of row r sits at chunk j ^ ((r >> 1) & 3), which keeps the shared-memory
 // writes at four wavefronts): half the TMA store operations of two 16-column boxes.  Needs a 2 KB box.
-__device__ __forceinline__ void store_row32_bf16(const OutMaps* om, uint8_t* xpose, int row0, int col0, int rows,
+__device__ __forceinline__ void store_row32_bf16(const OutMaps* om, uint8_t* xpose, int row0, int col0, bool live,
                                                  const uint32_t* w) {
   const int lane = threadIdx.x & 31;
   const int sw = (lane >> 1) & 3;
@@ -240,7 +255,7 @@ __device__ __forceinline__ void store_row32_bf16(const OutMaps* om, uint8_t* xpo
   uint4* mine = reinterpret_cast<uint4*>(xpose + lane * 64);
 #pragma unroll
   for (int j = 0; j < 4; ++j) mine[j ^ sw] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-  xpose_release(&om->out, xpose, col0, row0, rows);
+  xpose_release(&om->out, xpose, col0, row0, live);
 }
 
 // 32 consecutive output values of one row: bf16 (RNE) output and, when requested, the NVFP4
@@ -259,10 +274,10 @@ __device__ __forceinline__ void emit_row32(const GemmArgs& a, const OutMaps* om,
   }
   if (a.out != nullptr) {
     if constexpr (kBoxBytes >= 2048) {
-      store_row32_bf16(om, xpose, row0, col0, a.M, packed);
+      store_row32_bf16(om, xpose, row0, col0, row0 < a.M && col0 < a.n_out, packed);
     } else {
-      store_row16_bf16(om, xpose, row0, col0, a.M, packed);
-      store_row16_bf16(om, xpose, row0, col0 + 16, a.M, packed + 8);
+      store_row16_bf16(om, xpose, row0, col0, row0 < a.M && col0 < a.n_out, packed);
+      store_row16_bf16(om, xpose, row0, col0 + 16, row0 < a.M && col0 + 16 < a.n_out, packed + 8);
     }
   }
   if (a.q_codes != nullptr) {
@@ -296,7 +311,7 @@ __device__ __forceinline__ void emit_row32(const GemmArgs& a, const OutMaps* om,
     const int lane = threadIdx.x & 31;
     xpose_acquire();
     *reinterpret_cast<uint4*>(xpose + lane * 16) = make_uint4(words[0], words[1], words[2], words[3]);
-    xpose_release(&om->q_codes, xpose, col0 / 2, row0, a.M);
+    xpose_release(&om->q_codes, xpose, col0 / 2, row0, row0 < a.M && col0 < a.n_out);
     // the scale layout's rows end at the 128-row padding and its blocks at the 4-block padding of a row
     // (a ragged N's last tile reaches past both; its blocks up to the padding get zero scales)
     if (row < a.num_m_blocks * 128 && col0 / 16 < 4 * a.q_k_atoms)
@@ -492,7 +507,11 @@ __device__ __forceinline__ bool split_exchange(const GemmArgs& a, int tile, int 
     for (int i = 0; i < COLS / 4; ++i) part[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
     __threadfence();
     named_barrier_sync(1, 256);
+#ifdef NVFP4_TEST_HOOKS
+    if (et == 0 && !a.test_withhold_split_ready) atomicOr(&a.split_flags[tile], kSplitReady);
+#else
     if (et == 0) atomicOr(&a.split_flags[tile], kSplitReady);
+#endif
     return false;
   }
   if (et == 0) {

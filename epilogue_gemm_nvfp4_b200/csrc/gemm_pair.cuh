@@ -73,8 +73,13 @@ __device__ __forceinline__ PairUnit pair_unit(const GemmArgs& a, int u, int num_
   PairUnit w;
   const int split = u % a.splits;
   w.tile = u / a.splits;
-  w.mp = w.tile % a.num_m_pairs;
-  w.nb = w.tile / a.num_m_pairs;
+  if (a.n_fastest) {
+    w.nb = w.tile % a.num_n_blocks;
+    w.mp = w.tile / a.num_n_blocks;
+  } else {
+    w.mp = w.tile % a.num_m_pairs;
+    w.nb = w.tile / a.num_m_pairs;
+  }
   w.kb0 = split * num_kb / a.splits;
   w.kb1 = (split + 1) * num_kb / a.splits;
   return w;

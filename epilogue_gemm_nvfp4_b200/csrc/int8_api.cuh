@@ -130,6 +130,7 @@ nvfp4_status nvfp4_int8_linear(const nvfp4_int8_tensor* a, const nvfp4_int8_tens
   g.M = static_cast<int32_t>(M);
   g.N = static_cast<int32_t>(N);
   g.K = static_cast<int32_t>(K);
+  g.n_out = static_cast<int32_t>(n_out);
   g.num_m_blocks = static_cast<int32_t>((M + 127) / 128);
   g.num_n_blocks = static_cast<int32_t>(epi->kind == NVFP4_EPI_GATED_SILU ? (N / 2) / 128 : N / BN);
   g.num_tiles = g.num_m_blocks * g.num_n_blocks;
@@ -159,6 +160,7 @@ nvfp4_status nvfp4_int8_linear(const nvfp4_int8_tensor* a, const nvfp4_int8_tens
   g.out_amax_bits = reinterpret_cast<unsigned int*>(epi->out_amax);
   g.error_word = st->error_word;
   g.timeout_ns = wait_timeout_ns();
+  g.n_fastest = N <= M ? 1 : 0;  // keep the smaller operand resident in L2 (as nvfp4_linear does)
   g.splits = 1;
   g.num_units = g.num_tiles;
 

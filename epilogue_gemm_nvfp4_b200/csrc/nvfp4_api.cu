@@ -3,6 +3,7 @@
 // variable) and the per-stream split-K scratch of long-K GEMMs.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
 #include <map>
@@ -142,6 +143,11 @@ uint64_t wait_timeout_ns() {
   }();
   return ns;
 }
+
+#ifdef NVFP4_TEST_HOOKS
+// Test builds only (libnvfp4_testhooks.so): see nvfp4_test_withhold_split_ready.
+std::atomic<int> g_test_withhold_split_ready{0};
+#endif
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -407,6 +413,7 @@ nvfp4_status linear_impl(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvf
   g.M = static_cast<int32_t>(M);
   g.N = static_cast<int32_t>(N);
   g.K = static_cast<int32_t>(K);
+  g.n_out = static_cast<int32_t>(n_out);
   g.num_m_blocks = static_cast<int32_t>((M + 127) / 128);
   g.num_n_blocks = static_cast<int32_t>(epi->kind == NVFP4_EPI_GATED_SILU ? (N / 2) / 128 : (N + BN - 1) / BN);
   g.num_tiles = g.num_m_blocks * g.num_n_blocks;
@@ -439,6 +446,14 @@ nvfp4_status linear_impl(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvf
   g.out_amax_bits = reinterpret_cast<unsigned int*>(epi->out_amax);
   g.error_word = st->error_word;
   g.timeout_ns = wait_timeout_ns();
+#ifdef NVFP4_TEST_HOOKS
+  g.test_withhold_split_ready = g_test_withhold_split_ready.load();
+#endif
+  // Tile order: every wave of the persistent grid re-reads whichever operand the order sweeps, so the
+  // order keeps the smaller operand (same K: fewer rows) resident in L2 and streams the larger one from
+  // HBM once.  (Row blocks fastest re-read all of A every wave; for the 2048^2 down projection that is
+  // 117 MB of A per wave against a 126 MB L2.)  Which CTA computes a tile never changes its bits.
+  g.n_fastest = N <= M ? 1 : 0;
   g.splits = split_k_for(K, epi->kind);
   if (pair) g.num_tiles = g.num_m_pairs * g.num_n_blocks;  // 256 x 256 tiles of CTA pairs
   g.num_units = g.num_tiles * g.splits;
@@ -503,6 +518,14 @@ nvfp4_status nvfp4_linear_noalloc(const nvfp4_tensor* a, const nvfp4_tensor* w, 
 }
 
 size_t nvfp4_linear_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+#ifdef NVFP4_TEST_HOOKS
+// Test builds only, not declared in the public header: while `on` is non-zero, the split-K linears
+// launched afterwards withhold the first unit's ready bit, so that the second unit's bounded wait runs
+// out, the kernel gives up and nvfp4_get_device_error reports NVFP4_ERR_DEVICE_TIMEOUT.  This is how the
+// device-timeout path is exercised without faulting or hanging anything.
+NVFP4_API void nvfp4_test_withhold_split_ready(int32_t on) { g_test_withhold_split_ready.store(on != 0); }
+#endif
 
 nvfp4_status nvfp4_get_device_error(nvfp4_stream_t stream) {
   DeviceState* st;

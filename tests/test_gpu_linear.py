@@ -162,6 +162,51 @@ def test_gated_silu_with_requant_small(lib, M):
     assert torch.equal(q.codes, q3.codes) and torch.equal(q.scales, q3.scales)
 
 
+@pytest.mark.parametrize("kind,M,N,K", [("bias", 200, 144, 512), ("bias", 300, 400, 1024), ("resid_gate", 130, 400, 768),
+                                        ("bias", 257, 4624, 4608), ("resid_gate", 129, 4624, 1024),
+                                        ("bias", 130, 400, 32768)])
+def test_ragged_n(lib, kind, M, N, K):
+    """N a multiple of 16 but not of 128: 128-wide tiles whose last one reaches past N (the weight's rows
+    past N read as zeros, the epilogue reads no bias, residual or gate there, the stores are clipped)."""
+    assert B.tile_n(N, K, kind) == 128
+    if kind == "bias":
+        case = W.case_bias(M, N, K, seed=N + K, w_std=0.02 if K < 32768 else 0.005,
+                           x_dist="student_t" if K >= 32768 else "normal")
+        case.bias = W.to_bf16(np.random.default_rng(N).standard_normal(N).astype(np.float32))
+    else:
+        case = W.case_ffn_down(M, N=N, F=K, seed=N + K)
+    _, _, out = run_gpu(case)
+    assert out.shape == (M, N)
+    _, _, ref = run_oracle(case)
+    check(f32(out), ref["y"], f"ragged N {kind} {M}x{N}x{K}")
+
+
+def test_ragged_n_requant_and_amax(lib):
+    """The NVFP4 output and the output amax of a ragged-N bias GEMM: the fused codes equal nvfp4_quantize
+    of the kernel's own bf16 output bit for bit, padding scale bytes included (the last tile's blocks past
+    N land in the row's 4-block padding or past it), and the amax is the bf16 output's."""
+    M, N, K = 300, 400, 512
+    case = W.case_bias(M, N, K, seed=41, w_std=0.05)
+    aq, wq = B.quantize(case.x.cuda()), B.quantize(case.w.cuda())
+    bias = case.bias.cuda()
+    out = B.linear(aq, wq, "bias", bias=bias)
+    g_out = bf16_absmax(out) / 2688.0
+    # GEMM NVFP4 outputs need 16-byte code rows: 400 columns are 200 bytes, so the rows are padded to 208
+    codes = torch.zeros(M, 208, dtype=torch.uint8, device="cuda")[:, : N // 2]
+    q = B.QTensor(codes, torch.full((B.scale_bytes(M, N),), 0x55, dtype=torch.uint8, device="cuda"),
+                  torch.full((1,), g_out, dtype=torch.float32, device="cuda"), M, N)
+    # (the scales start as 0x55: the fused requant must write every scale byte, padding included, as the
+    # quantiser does)
+    amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+    out2 = B.linear(aq, wq, "bias", bias=bias, out_fp4=q, out_amax=amax)
+    B.check_device_error()
+    assert torch.equal(out, out2)
+    q2 = B.quantize(out, g=g_out)
+    torch.cuda.synchronize()
+    assert torch.equal(q.codes, q2.codes) and torch.equal(q.scales, q2.scales)
+    assert float(amax.item()) == bf16_absmax(out)
+
+
 def test_tile_n_128_path_and_k_tail(lib):
     # N = 384 forces 128-wide tiles (two TMEM accumulators); K = 320 leaves a one-MMA tail stage
     case = W.case_bias(515, 384, 320, seed=9, w_std=0.05)
