@@ -761,31 +761,31 @@ __global__ void __launch_bounds__(512, 1)
           const int ks = min(C::KSTEPS, args.k_steps - kb * C::KSTEPS);
           const uint32_t t_sf = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + C::SF_COL0 + stage * C::SF_COLS;
           // slot column order: A steps 0..KSTEPS-1 (4 columns each), then for each step k the weight's
-          // 128-row blocks j = 0 .. BN/128-1 (4 columns each)
-  #pragma unroll
-          for (int grp = 0; grp < NV / 2; ++grp) {
-            uint32_t v[8];
-  #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int idx = grp * 2 + h;
-              int k;
-              const uint8_t* src;
-              if (idx < C::KSTEPS) {
-                k = idx;
-                src = ssfa + k * C::SF_ATOM_BYTES;
-              } else {
-                k = (idx - C::KSTEPS) / (BN / 128);
-                src = ssfb + ((idx - C::KSTEPS) % (BN / 128)) * C::KSTEPS * C::SF_ATOM_BYTES + k * C::SF_ATOM_BYTES;
-              }
-              uint4 x = make_uint4(0, 0, 0, 0);
-              if (k < ks) x = *reinterpret_cast<const uint4*>(src + lane * 16);
-              v[4 * h + 0] = x.x;
-              v[4 * h + 1] = x.y;
-              v[4 * h + 2] = x.z;
-              v[4 * h + 3] = x.w;
+          // 128-row blocks j = 0 .. BN/128-1 (4 columns each).  The slot's NV vectors (16 bytes each) are
+          // gathered, then written with the widest stores (one 32- and one 16-column tcgen05.st for a
+          // 48-column slot, one 32-column store for a 32-column slot).
+          uint32_t v[4 * NV];
+#pragma unroll
+          for (int idx = 0; idx < NV; ++idx) {
+            int k;
+            const uint8_t* src;
+            if (idx < C::KSTEPS) {
+              k = idx;
+              src = ssfa + k * C::SF_ATOM_BYTES;
+            } else {
+              k = (idx - C::KSTEPS) / (BN / 128);
+              src = ssfb + ((idx - C::KSTEPS) % (BN / 128)) * C::KSTEPS * C::SF_ATOM_BYTES + k * C::SF_ATOM_BYTES;
             }
-            tmem_st_32x32b_x8(t_sf + grp * 8, v);
+            uint4 x = make_uint4(0, 0, 0, 0);
+            if (k < ks) x = *reinterpret_cast<const uint4*>(src + lane * 16);
+            v[4 * idx + 0] = x.x;
+            v[4 * idx + 1] = x.y;
+            v[4 * idx + 2] = x.z;
+            v[4 * idx + 3] = x.w;
           }
+          static_assert(NV == 12 || NV == 8, "a slot is 48 or 32 columns");
+          tmem_st_32x32b_x32(t_sf, v);
+          if constexpr (NV == 12) tmem_st_32x32b_x16(t_sf + 32, v + 32);
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();

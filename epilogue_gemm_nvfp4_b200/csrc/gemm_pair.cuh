@@ -285,33 +285,33 @@ __global__ void __launch_bounds__(512, 1) __cluster_dims__(2, 1, 1)
         const uint8_t* ssfb = ssfa + C::SFA_BYTES;
         const int ks = min(C::KSTEPS, args.k_steps - kb * C::KSTEPS);
         const uint32_t t_sf = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + C::SF_COL0 + stage * C::SF_COLS;
+        // gather the slot's NV vectors (16 bytes each) into registers, then write them with the widest
+        // stores: one 32- and one 16-column tcgen05.st for the 48-column slot
+        uint32_t v[4 * NV];
 #pragma unroll
-        for (int grp = 0; grp < NV / 2; ++grp) {
-          uint32_t v[8];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int idx = grp * 2 + h;
-            int k;
-            bool have;
-            const uint8_t* src;
-            if (idx < C::KSTEPS) {
-              k = idx;
-              have = a_rows;
-              src = ssfa + k * C::SF_ATOM_BYTES;
-            } else {
-              k = (idx - C::KSTEPS) / (C::BN / 128);
-              have = true;
-              src = ssfb + ((idx - C::KSTEPS) % (C::BN / 128)) * C::KSTEPS * C::SF_ATOM_BYTES + k * C::SF_ATOM_BYTES;
-            }
-            uint4 x = make_uint4(0, 0, 0, 0);
-            if (have && k < ks) x = *reinterpret_cast<const uint4*>(src + lane * 16);
-            v[4 * h + 0] = x.x;
-            v[4 * h + 1] = x.y;
-            v[4 * h + 2] = x.z;
-            v[4 * h + 3] = x.w;
+        for (int idx = 0; idx < NV; ++idx) {
+          int k;
+          bool have;
+          const uint8_t* src;
+          if (idx < C::KSTEPS) {
+            k = idx;
+            have = a_rows;
+            src = ssfa + k * C::SF_ATOM_BYTES;
+          } else {
+            k = (idx - C::KSTEPS) / (C::BN / 128);
+            have = true;
+            src = ssfb + ((idx - C::KSTEPS) % (C::BN / 128)) * C::KSTEPS * C::SF_ATOM_BYTES + k * C::SF_ATOM_BYTES;
           }
-          tmem_st_32x32b_x8(t_sf + grp * 8, v);
+          uint4 x = make_uint4(0, 0, 0, 0);
+          if (have && k < ks) x = *reinterpret_cast<const uint4*>(src + lane * 16);
+          v[4 * idx + 0] = x.x;
+          v[4 * idx + 1] = x.y;
+          v[4 * idx + 2] = x.z;
+          v[4 * idx + 3] = x.w;
         }
+        static_assert(NV == 12, "a slot is 48 columns: one 32- and one 16-column store");
+        tmem_st_32x32b_x32(t_sf, v);
+        tmem_st_32x32b_x16(t_sf + 32, v + 32);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
