@@ -82,6 +82,13 @@ def test_argument_checks_return_before_any_launch(lib):
     q = _tensor(256, 256)
     gs = B.CEpilogue(kind=B.EPI_GATED_SILU, out_nvfp4=1)
     assert lin(a, w, gs, q=ctypes.byref(_tensor(256, 512))) == B.ERR_INVALID_ARG           # out_fp4 not [M, N/2]
+    # empty and oversized problems: M = 0 is a valid call that launches nothing (so it succeeds even
+    # without a device); a dimension past 2^30 is refused
+    assert lin(_tensor(0, 512), w, desc, out=0x10000) == B.OK
+    big = 1 << 30
+    assert lin(_tensor(big + 1, 512), w, desc) == B.ERR_UNSUPPORTED_SHAPE                 # M > 2^30
+    assert lin(_tensor(256, 512), _tensor(big + 256, 512), desc, ld=big + 256) == B.ERR_UNSUPPORTED_SHAPE
+    assert lin(_tensor(256, big + 64), _tensor(512, big + 64), desc) == B.ERR_UNSUPPORTED_SHAPE
     # quantise / dequantise / amax
     t = _tensor(4, 512)
     assert lib.nvfp4_quantize(None, 4, 512, 512, 1, ctypes.byref(t), None) == B.ERR_INVALID_ARG

@@ -136,3 +136,30 @@ def test_fake_quantize_static_scale_and_strides(lib):
     assert out.data_ptr() == y.data_ptr()
     ref_y, _ = O.fake_quantize(f32(base)[:, 32:32 + 512], np.float32(g))
     np.testing.assert_array_equal(f32(out), ref_y)
+
+
+def test_empty_inputs_through_the_abi(lib):
+    """rows == 0 / M == 0: the quantiser writes no codes and its dynamic scale is 1 (the all-zero rule), the
+    scale padding rows are zero, and the fused linear returns without touching its output.  Called through
+    the C ABI with real buffers (torch reports a null data pointer for a tensor with no elements)."""
+    import ctypes
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    x = torch.ones((1, 512), dtype=torch.bfloat16, device="cuda")
+    codes = torch.full((1, 256), 0x77, dtype=torch.uint8, device="cuda")
+    scales = torch.full((B.scale_bytes(0, 512) or 1,), 0x55, dtype=torch.uint8, device="cuda")
+    g = torch.zeros(1, dtype=torch.float32, device="cuda")
+    t = B.CTensor(codes.data_ptr(), scales.data_ptr(), g.data_ptr(), 0, 512, 256)
+    assert lib.nvfp4_quantize(x.data_ptr(), 0, 512, 512, 1, ctypes.byref(t), stream) == B.OK
+    torch.cuda.synchronize()
+    assert g.item() == 1.0
+    assert torch.all(codes == 0x77)          # no row to encode
+    # the fused linear with an empty activation: nothing is launched, the output keeps its contents
+    wq = B.quantize(rand_bf16(256, 512, 3).cuda())
+    out = torch.full((1, 256), 7.0, dtype=torch.bfloat16, device="cuda")
+    desc = B.make_epilogue("bias")
+    cw = wq.c()
+    assert lib.nvfp4_linear(ctypes.byref(t), ctypes.byref(cw), ctypes.byref(desc), out.data_ptr(), 256, None,
+                            stream) == B.OK
+    torch.cuda.synchronize()
+    assert torch.all(out == 7.0)
+    B.check_device_error()
