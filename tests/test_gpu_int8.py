@@ -1,7 +1,8 @@
 """GPU parity of the W8A8 INT8 path through the C ABI: the per-row quantiser must equal the oracle byte for
 byte; the linear's integer products are exact, so its output differs from the oracle's fp64 value only by
 the fp32 scaling and the bf16 rounding (half a bf16 step plus a few fp32 roundings), except where the
-epilogue itself approximates (the hardware tanh of the gated SiLU)."""
+epilogue itself approximates (the fast exponential and division of the gated SiLU, the head norm's
+reciprocal square root)."""
 import numpy as np
 import pytest
 import torch
@@ -82,7 +83,8 @@ def test_int8_linear_resid_gate(lib):
 
 
 def test_int8_linear_qknorm_and_gated_silu(lib):
-    """Nonlinear epilogues: within 3e-3 normwise of the oracle (the gated SiLU uses the hardware tanh)."""
+    """Nonlinear epilogues: within 3e-3 normwise of the oracle (fast exponential, division and reciprocal
+    square root in the epilogue)."""
     M, K = 130, 512
     rng = np.random.default_rng(7)
     gq, gk = W.to_bf16(W.uniform(rng, (256,), 0.5, 1.5)), W.to_bf16(W.uniform(rng, (256,), 0.5, 1.5))
