@@ -7,14 +7,16 @@
 // therefore receives half of the B codes it would load for a one-CTA 128 x 256 tile: a third less
 // TMA and shared-memory traffic per FLOP, and a stage of 38 KB instead of 54 KB (5 stages).
 //
-// Roles per CTA (as in the one-CTA kernel):
-//   warp 0     producer: its A box and its half of B with the paired TMA form, whose bytes are
-//              counted on the leader's `full` barrier (the leader arms it for both CTAs' bytes); its
-//              scale atoms (A's for its own rows, B's for all 256 rows) with bulk copies on its own
-//              `sf_landed`.  No multicast loads.
-//   warp 1     leader only: the MMA issuer; commits go to both CTAs' `empty` / `acc_full`.
+// Roles per CTA:
+//   warp 0     producer: its A box, its half of B and its scale atoms (A's for its own rows, B's for
+//              all 256 rows), all with the paired TMA form, whose bytes are counted on the leader's
+//              `full` barrier (the leader arms it for both CTAs' bytes).  No multicast loads.
+//   warp 1     leader only: the MMA issuer, the whole warp converged with one elected lane issuing.
+//              Per stage it copies the stage's twelve scale atoms from both CTAs' shared memory into
+//              their TMEM scale slot (tcgen05.cp, which the tensor pipe runs in order with the MMAs
+//              that follow), then issues the four MMAs; commits go to both CTAs' `empty` / `acc_full`.
 //   warp 2     TMEM allocation (paired form).
-//   warps 4-7  scale stagers into this CTA's TMEM, then an arrival on the leader's `full`.
+//   warps 3-7  idle.
 //   warps 8-15 epilogue of this CTA's 128 rows; the accumulator release is an arrival on the
 //              leader's `acc_empty` (16 arrivals: 8 warps per CTA).
 // 128-wide tiles stay on the one-CTA kernel.  Split-K units exchange partial sums per (pair tile,
@@ -53,13 +55,19 @@ struct GemmPairCfg {
   static constexpr int SMEM_BYTES = AUX_BYTES + 1023 + STAGES * STAGE_BYTES + EPI_WARPS * XPOSE_BYTES;
   static constexpr uint32_t IDESC = idesc_nvf4(2 * BM, BN);
   static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");
-  static_assert(SF_COLS % 8 == 0, "scale slot is written 8 columns at a time");
+  static_assert(SF_COLS % 4 == 0, "a scale atom fills four TMEM columns");
   static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
   static_assert(STAGE_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
   static_assert((3 * STAGES + 5) * 8 + 16 <= SS_OFFSET, "barrier area");
   static_assert((SMEM_LIMIT >> 4) < (1 << 14), "operand descriptors advance by adds inside the 14-bit address field");
   // the epilogue and its column split are those of the one-CTA 256-wide tile
   static_assert(GemmCfg<256>::EPI_WARPS == EPI_WARPS, "epilogue");
+};
+
+// TMA maps over the block-scale bytes viewed as rows of one 512-byte atom (128 x uint32): a box of
+// four rows is the four atoms of one 128-row block for one stage.
+struct ScaleMaps {
+  CUtensorMap sfa, sfb;
 };
 
 struct PairUnit {
@@ -89,14 +97,14 @@ __device__ __forceinline__ PairUnit pair_unit(const GemmArgs& a, int u, int num_
 template <int KIND, bool kSplit>
 __global__ void __launch_bounds__(512, 1) __cluster_dims__(2, 1, 1)
     nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                           const __grid_constant__ OutMaps out_maps, const __grid_constant__ GemmArgs args) {
+                           const __grid_constant__ ScaleMaps sf_maps, const __grid_constant__ OutMaps out_maps,
+                           const __grid_constant__ GemmArgs args) {
   using C = GemmPairCfg;
   using E = Epilogue<256, KIND, C::XPOSE_BYTES>;
   extern __shared__ uint8_t smem_raw[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* sf_landed = empty + C::STAGES;
-  uint64_t* acc_full = sf_landed + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -116,10 +124,9 @@ __global__ void __launch_bounds__(512, 1) __cluster_dims__(2, 1, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      // leader's copy: its expect-tx arrival (for both CTAs' code bytes) + 4 stager warps per CTA
-      mbar_init(&full[s], 1 + 8);
+      // leader's copy: its expect-tx arrival for both CTAs' bytes
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&sf_landed[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -133,6 +140,8 @@ __global__ void __launch_bounds__(512, 1) __cluster_dims__(2, 1, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmap_a);
     prefetch_tensormap(&tmap_b);
+    prefetch_tensormap(&sf_maps.sfa);
+    prefetch_tensormap(&sf_maps.sfb);
     if (args.out != nullptr) prefetch_tensormap(&out_maps.out);
     if (args.q_codes != nullptr) prefetch_tensormap(&out_maps.q_codes);
   }
@@ -154,175 +163,124 @@ __global__ void __launch_bounds__(512, 1) __cluster_dims__(2, 1, 1)
         // ---------------------------------------------------------------- TMA producer (both CTAs)
         int stage = 0;
         uint32_t phase = 0;
-        uint32_t armed_mask = 0, armed_parity = 0;
         bool ok = true;
         for (int u = cluster; ok && u < args.num_units; u += num_clusters) {
           const PairUnit pu = pair_unit(args, u, num_kb);
-          const int mb = 2 * pu.mp + static_cast<int>(rank);  // this CTA's 128-row block of A
-          const bool a_rows = mb < args.num_m_blocks;         // false: the block lies wholly past M
+          // this CTA's 128-row block of A; a block wholly past M reads zeros (codes and scales)
+          const int mb = 2 * pu.mp + static_cast<int>(rank);
           for (int kb = pu.kb0; kb < pu.kb1; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.timeout_ns)) {
               ok = false;
               break;
             }
-            const int ks = min(C::KSTEPS, args.k_steps - kb * C::KSTEPS);
-            const uint32_t sf_bytes = static_cast<uint32_t>(ks) * 512u;
             uint8_t* sa = ring + stage * C::STAGE_BYTES;
             uint8_t* sb = sa + C::A_BYTES;
             uint8_t* ssfa = sb + C::B_BYTES;
             uint8_t* ssfb = ssfa + C::SFA_BYTES;
-            mbar_arrive_expect_tx(&sf_landed[stage], sf_bytes * ((a_rows ? 1 : 0) + C::BN / 128));
-            if (a_rows)
-              bulk_load(ssfa, args.sfa + (static_cast<int64_t>(mb) * args.k_atoms + kb * C::KSTEPS) * 512, sf_bytes,
-                        &sf_landed[stage]);
-#pragma unroll
-            for (int j = 0; j < C::BN / 128; ++j)
-              bulk_load(ssfb + j * C::KSTEPS * C::SF_ATOM_BYTES,
-                        args.sfb + (static_cast<int64_t>(b_row0<256, KIND>(args, pu.nb, j) / 128) * args.k_atoms +
-                                    kb * C::KSTEPS) * 512,
-                        sf_bytes, &sf_landed[stage]);
             const uint32_t leader_full = cluster_addr(&full[stage], 0);
-            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (C::A_BYTES + C::B_BYTES));
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
             tma_load_2d_pair(sa, &tmap_a, leader_full, kb * C::BK_BYTES, mb * C::BM);
             tma_load_2d_pair(sb, &tmap_b, leader_full, kb * C::BK_BYTES,
                              b_row0<256, KIND>(args, pu.nb, static_cast<int>(rank)));
-            armed_mask |= 1u << stage;
-            armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+            // scale atoms: rows of the scale maps are atoms, ordered along K within a 128-row block;
+            // a K tail loads the next atoms too, which no MMA reads
+            tma_load_2d_pair(ssfa, &sf_maps.sfa, leader_full, 0, mb * args.k_atoms + kb * C::KSTEPS);
+#pragma unroll
+            for (int j = 0; j < C::BN / 128; ++j)
+              tma_load_2d_pair(ssfb + j * C::KSTEPS * C::SF_ATOM_BYTES, &sf_maps.sfb, leader_full, 0,
+                               (b_row0<256, KIND>(args, pu.nb, j) / 128) * args.k_atoms + kb * C::KSTEPS);
             if (++stage == C::STAGES) {
               stage = 0;
               phase ^= 1u;
             }
           }
         }
+        // every box this CTA loads is counted on the leader's `full`, which the leader's MMA thread
+        // consumes before the final cluster barrier
         if (!ok) raise_device_error(args.error_word, kErrTimeout, abort_flag);
-        // this CTA's scale copies must land before its shared memory is released; its code boxes are
-        // counted on the leader's `full`, which the leader's MMA thread consumed before the final
-        // cluster barrier
-        for (int s = 0; s < C::STAGES; ++s)
-          if (armed_mask & (1u << s)) mbar_wait(&sf_landed[s], (armed_parity >> s) & 1u, never_abort, args.timeout_ns);
       }
       __syncwarp();
     } else if (warp == 1) {
-      if (lane == 0 && rank == 0) {
+      if (rank == 0) {
         // ---------------------------------------------------------------- MMA issuer (leader)
+        // The whole warp runs this loop converged and one elected lane issues each tcgen05 instruction;
+        // every operand is warp-uniform (the TMEM base is broadcast from lane 0 so that the compiler
+        // can prove it), and each wait's outcome is agreed by a vote.
+        const uint32_t t_base = __shfl_sync(0xFFFFFFFFu, tmem_base, 0);
         constexpr uint64_t kStageDesc = C::STAGE_BYTES >> 4;
         const uint64_t a_desc0 = desc_kmajor_swizzled<C::BK_BYTES>(smem_u32(ring));
         const uint64_t b_desc_off = C::A_BYTES >> 4;
-        const uint32_t sf_col0 = tmem_base + C::SF_COL0;
+        const uint64_t sf_desc0 = desc_scale_atom(smem_u32(ring + C::A_BYTES + C::B_BYTES));
+        const uint32_t sf_col0 = t_base + C::SF_COL0;
         int stage = 0;
         uint32_t phase = 0;
         uint64_t a_desc = a_desc0;
+        uint64_t sf_desc = sf_desc0;
         uint32_t sfa_t = sf_col0;
         uint32_t aphase = 0;
         bool ok = true;
         for (int u = cluster; ok && u < args.num_units; u += num_clusters) {
           const PairUnit pu = pair_unit(args, u, num_kb);
-          if (!mbar_wait(&acc_empty[0], aphase ^ 1u, abort_flag, args.timeout_ns)) {
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_empty[0], aphase ^ 1u, abort_flag, args.timeout_ns))) {
             ok = false;
             break;
           }
           tc_fence_after();
           uint32_t accumulate = 0;
           for (int kb = pu.kb0; kb < pu.kb1; ++kb) {
-            if (!mbar_wait(&full[stage], phase, abort_flag, args.timeout_ns)) {
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[stage], phase, abort_flag, args.timeout_ns))) {
               ok = false;
               break;
             }
             tc_fence_after();
+            // scale slot: atom v (A's atoms k = 0..3, then B's atoms k = 0..3 of both 128-row blocks,
+            // interleaved by block) to columns 4v..4v+3, where the MMAs below read them
+#pragma unroll
+            for (int v = 0; v < C::SF_COLS / 4; ++v) {
+              const int off = v < C::KSTEPS ? v * C::SF_ATOM_BYTES
+                                            : C::SFA_BYTES + ((v - C::KSTEPS) % (C::BN / 128)) * C::KSTEPS * C::SF_ATOM_BYTES +
+                                                  ((v - C::KSTEPS) / (C::BN / 128)) * C::SF_ATOM_BYTES;
+              tc_cp_pair_32x128b_warpx4_warp(sfa_t + 4 * v, sf_desc + (off >> 4));
+            }
             const uint64_t b_desc = a_desc + b_desc_off;
             const uint32_t sfb_t = sfa_t + C::SFA_COLS;
             if (kb * C::KSTEPS + C::KSTEPS <= args.k_steps) {
 #pragma unroll
               for (int k = 0; k < C::KSTEPS; ++k)
-                tc_mma_nvf4_pair(tmem_base, a_desc + 2 * k, b_desc + 2 * k, C::IDESC, accumulate | k, sfa_t + k * 4,
-                                 sfb_t + k * (C::BN / 32));
+                tc_mma_nvf4_pair_warp(t_base, a_desc + 2 * k, b_desc + 2 * k, C::IDESC, accumulate | k, sfa_t + k * 4,
+                                      sfb_t + k * (C::BN / 32));
             } else {
               const int ks = args.k_steps - kb * C::KSTEPS;
               for (int k = 0; k < ks; ++k)
-                tc_mma_nvf4_pair(tmem_base, a_desc + 2 * k, b_desc + 2 * k, C::IDESC, accumulate | k, sfa_t + k * 4,
-                                 sfb_t + k * (C::BN / 32));
+                tc_mma_nvf4_pair_warp(t_base, a_desc + 2 * k, b_desc + 2 * k, C::IDESC, accumulate | k, sfa_t + k * 4,
+                                      sfb_t + k * (C::BN / 32));
             }
             accumulate = 1;
-            tc_commit_pair(&empty[stage], 0x3);
+            tc_commit_pair_warp(&empty[stage], 0x3);
             if (++stage == C::STAGES) {
               stage = 0;
               phase ^= 1u;
               a_desc = a_desc0;
+              sf_desc = sf_desc0;
               sfa_t = sf_col0;
             } else {
               a_desc += kStageDesc;
+              sf_desc += kStageDesc;
               sfa_t += C::SF_COLS;
             }
           }
           if (!ok) break;
-          tc_commit_pair(&acc_full[0], 0x3);
+          tc_commit_pair_warp(&acc_full[0], 0x3);
           aphase ^= 1u;
         }
-        if (!ok) raise_device_error(args.error_word, kErrTimeout, abort_flag);
-        tc_commit_pair(drain, 0x1);
+        if (!ok && lane == 0) raise_device_error(args.error_word, kErrTimeout, abort_flag);
+        tc_commit_pair_warp(drain, 0x1);
         mbar_wait(drain, 0, never_abort, args.timeout_ns);
       }
       __syncwarp();
     }
   } else if (warp < 8) {
-    regs_decrease<64>();
-    // ------------------------------------------------------------------ scale stagers (both CTAs)
-    const int q = warp & 3;
-    constexpr int NV = C::SF_COLS / 4;
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int u = cluster; ok && u < args.num_units; u += num_clusters) {
-      const PairUnit pu = pair_unit(args, u, num_kb);
-      const bool a_rows = 2 * pu.mp + static_cast<int>(rank) < args.num_m_blocks;
-      for (int kb = pu.kb0; kb < pu.kb1; ++kb) {
-        const bool got = mbar_wait(&sf_landed[stage], phase, abort_flag, args.timeout_ns);
-        if (!__all_sync(0xFFFFFFFFu, got)) {
-          ok = false;
-          break;
-        }
-        const uint8_t* ssfa = ring + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
-        const uint8_t* ssfb = ssfa + C::SFA_BYTES;
-        const int ks = min(C::KSTEPS, args.k_steps - kb * C::KSTEPS);
-        const uint32_t t_sf = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + C::SF_COL0 + stage * C::SF_COLS;
-        // gather the slot's NV vectors (16 bytes each) into registers, then write them with the widest
-        // stores: one 32- and one 16-column tcgen05.st for the 48-column slot
-        uint32_t v[4 * NV];
-#pragma unroll
-        for (int idx = 0; idx < NV; ++idx) {
-          int k;
-          bool have;
-          const uint8_t* src;
-          if (idx < C::KSTEPS) {
-            k = idx;
-            have = a_rows;
-            src = ssfa + k * C::SF_ATOM_BYTES;
-          } else {
-            k = (idx - C::KSTEPS) / (C::BN / 128);
-            have = true;
-            src = ssfb + ((idx - C::KSTEPS) % (C::BN / 128)) * C::KSTEPS * C::SF_ATOM_BYTES + k * C::SF_ATOM_BYTES;
-          }
-          uint4 x = make_uint4(0, 0, 0, 0);
-          if (have && k < ks) x = *reinterpret_cast<const uint4*>(src + lane * 16);
-          v[4 * idx + 0] = x.x;
-          v[4 * idx + 1] = x.y;
-          v[4 * idx + 2] = x.z;
-          v[4 * idx + 3] = x.w;
-        }
-        static_assert(NV == 12, "a slot is 48 columns: one 32- and one 16-column store");
-        tmem_st_32x32b_x32(t_sf, v);
-        tmem_st_32x32b_x16(t_sf + 32, v + 32);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(cluster_addr(&full[stage], 0));
-        if (++stage == C::STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-    }
-    if (!ok && lane == 0) raise_device_error(args.error_word, kErrTimeout, abort_flag);
+    regs_decrease<64>();  // idle: the scale atoms reach TMEM through the MMA thread's copies
   } else {
     regs_increase<192>();
     // ------------------------------------------------------------------ epilogue (both CTAs)

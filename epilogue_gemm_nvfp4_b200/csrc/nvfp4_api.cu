@@ -202,6 +202,23 @@ nvfp4_status make_code_map(CUtensorMap* map, const nvfp4_tensor* t) {
   return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+// 2-D TMA descriptor over a tensor's block-scale bytes viewed as rows of one 512-byte atom (128 x
+// uint32, unswizzled): row b * k_atoms + k is atom k of 128-row block b.  A box is four atoms, the
+// scales of one 128-row block for one stage of K; rows past the last block read as zeros.
+nvfp4_status make_scale_map(CUtensorMap* map, const nvfp4_tensor* t) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return NVFP4_ERR_CUDA;
+  const int64_t atoms = (t->rows + 127) / 128 * k_atoms_of(t->cols);
+  cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(atoms)};
+  cuuint64_t strides[1] = {512};
+  cuuint32_t box[2] = {128, static_cast<cuuint32_t>(kStageKSteps)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, t->scales, dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
 // TMA store maps of the fused linear's outputs, in the boxes the epilogue writes (32 rows of one warp):
 // bf16 output `box_cols` (16 or 32) columns wide with the 32- or 64-byte swizzle of its shared-memory
 // box, E2M1 codes 16 bytes wide unswizzled.  A map stays zeroed when its output is not requested (the
@@ -263,8 +280,8 @@ bool pair_kernel_enabled() {
 }
 
 template <int KIND, bool kSplit>
-nvfp4_status launch_gemm_pair_as(DeviceState* st, const CUtensorMap& ma, const CUtensorMap& mb, const OutMaps& om,
-                                 const GemmArgs& args, cudaStream_t stream) {
+nvfp4_status launch_gemm_pair_as(DeviceState* st, const CUtensorMap& ma, const CUtensorMap& mb, const ScaleMaps& sm,
+                                 const OutMaps& om, const GemmArgs& args, cudaStream_t stream) {
   using C = GemmPairCfg;
   auto kernel = nvfp4_gemm_pair_kernel<KIND, kSplit>;
   int clusters = 0;
@@ -287,18 +304,18 @@ nvfp4_status launch_gemm_pair_as(DeviceState* st, const CUtensorMap& ma, const C
     clusters = cached;
   }
   const int grid_clusters = args.num_units < clusters ? args.num_units : clusters;
-  kernel<<<2 * grid_clusters, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, om, args);
+  kernel<<<2 * grid_clusters, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, sm, om, args);
   return launch_status();
 }
 
 template <int KIND>
-nvfp4_status launch_gemm_pair(DeviceState* st, const CUtensorMap& ma, const CUtensorMap& mb, const OutMaps& om,
-                              const GemmArgs& args, cudaStream_t stream) {
+nvfp4_status launch_gemm_pair(DeviceState* st, const CUtensorMap& ma, const CUtensorMap& mb, const ScaleMaps& sm,
+                              const OutMaps& om, const GemmArgs& args, cudaStream_t stream) {
   if constexpr (KIND == kEpiQkNorm) {
-    return launch_gemm_pair_as<KIND, false>(st, ma, mb, om, args, stream);  // never split
+    return launch_gemm_pair_as<KIND, false>(st, ma, mb, sm, om, args, stream);  // never split
   } else {
-    return args.splits > 1 ? launch_gemm_pair_as<KIND, true>(st, ma, mb, om, args, stream)
-                           : launch_gemm_pair_as<KIND, false>(st, ma, mb, om, args, stream);
+    return args.splits > 1 ? launch_gemm_pair_as<KIND, true>(st, ma, mb, sm, om, args, stream)
+                           : launch_gemm_pair_as<KIND, false>(st, ma, mb, sm, om, args, stream);
   }
 }
 
@@ -477,11 +494,14 @@ nvfp4_status linear_impl(const nvfp4_tensor* a, const nvfp4_tensor* w, const nvf
     if (cudaMemsetAsync(ws, 0, static_cast<size_t>(exch_slots) * 4, s) != cudaSuccess) return NVFP4_ERR_CUDA;
   }
   if (pair) {
+    ScaleMaps sm;
+    if (nvfp4_status e = make_scale_map(&sm.sfa, a)) return e;
+    if (nvfp4_status e = make_scale_map(&sm.sfb, w)) return e;
     switch (epi->kind) {
-      case NVFP4_EPI_BIAS: return launch_gemm_pair<kEpiBias>(st, ma, mb, om, g, s);
-      case NVFP4_EPI_RESID_GATE: return launch_gemm_pair<kEpiResidGate>(st, ma, mb, om, g, s);
-      case NVFP4_EPI_QKNORM: return launch_gemm_pair<kEpiQkNorm>(st, ma, mb, om, g, s);
-      case NVFP4_EPI_GATED_SILU: return launch_gemm_pair<kEpiGatedSilu>(st, ma, mb, om, g, s);
+      case NVFP4_EPI_BIAS: return launch_gemm_pair<kEpiBias>(st, ma, mb, sm, om, g, s);
+      case NVFP4_EPI_RESID_GATE: return launch_gemm_pair<kEpiResidGate>(st, ma, mb, sm, om, g, s);
+      case NVFP4_EPI_QKNORM: return launch_gemm_pair<kEpiQkNorm>(st, ma, mb, sm, om, g, s);
+      case NVFP4_EPI_GATED_SILU: return launch_gemm_pair<kEpiGatedSilu>(st, ma, mb, sm, om, g, s);
     }
     return NVFP4_ERR_INVALID_ARG;
   }

@@ -212,25 +212,44 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
+// The paired tcgen05 issue forms below are warp-collective: the whole warp executes them converged,
+// with warp-uniform operands, and one elected lane issues the instruction.  Issued from a single lane
+// inside a divergent branch, the same instructions cost the issuing thread several times longer,
+// since their operands must then be moved into the uniform datapath at every issue.
+
 // D[tmem] (+)= (A * SFA) x (B * SFB)^T over the CTA pair: M = 256 (128 rows of A in each CTA's shared
 // memory), N from the instruction descriptor (N/2 rows of B in each CTA's), K = 64.  Each CTA's TMEM
 // holds its 128 rows of D and the scales its rows use.
-__device__ __forceinline__ void tc_mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                                 uint32_t accumulate, uint32_t sfa_tmem, uint32_t sfb_tmem) {
+__device__ __forceinline__ void tc_mma_nvf4_pair_warp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                      uint32_t accumulate, uint32_t sfa_tmem, uint32_t sfb_tmem) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+      "@e tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
           d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
 
-// Arrive once on the barrier at `bar`'s offset in every CTA of `cta_mask` when the paired tcgen05
-// operations this thread issued before have completed.
-__device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+// Paired shared memory -> TMEM copy on the tensor pipe: in each CTA of the pair, 32 rows x 128 bits
+// from this CTA's shared memory (described by `sdesc`) to four TMEM columns at `taddr`, replicated into
+// all four 32-lane sub-partitions.  It executes in issue order with the MMAs issued after it, and a
+// later tcgen05.commit covers its shared-memory read.
+__device__ __forceinline__ void tc_cp_pair_32x128b_warpx4_warp(uint32_t taddr, uint64_t sdesc) {
   asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr),
+      "l"(sdesc)
+      : "memory");
+}
+
+// Arrive once on the barrier at `bar`'s offset in every CTA of `cta_mask` when the paired tcgen05
+// operations issued before have completed.
+__device__ __forceinline__ void tc_commit_pair_warp(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n\t}" ::"r"(
           smem_u32(bar)),
       "h"(cta_mask)
       : "memory");
@@ -338,6 +357,19 @@ __device__ __forceinline__ uint64_t desc_kmajor_swizzled(uint32_t saddr) {
   d |= static_cast<uint64_t>(1) << 46;                              // descriptor version for sm_100
   d |= static_cast<uint64_t>(kRowBytes == 128 ? 2 : 4) << 61;       // layout: 128- / 64-byte swizzle
   return d;
+}
+
+// Shared-memory matrix descriptor of one 512-byte scale atom as the source of a 32x128b tcgen05.cp:
+// 32 rows of 16 bytes, stored densely and unswizzled, i.e. four 8-row core matrices of 128 bytes
+// each.  The stride offset steps to the next core matrix; a row is a single core matrix wide, so the
+// leading offset is unused.
+__device__ __forceinline__ uint64_t desc_scale_atom(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);             // start address, 16-byte units
+  d |= static_cast<uint64_t>(1) << 16;                              // leading offset (unused)
+  d |= static_cast<uint64_t>(128 >> 4) << 32;                       // stride offset: next 8 rows
+  d |= static_cast<uint64_t>(1) << 46;                              // descriptor version for sm_100
+  return d;                                                         // layout type 0: no swizzle
 }
 
 // Instruction descriptor for kind::mxf4nvf4: E2M1 x E2M1, UE4M3 scales, fp32 accumulator,
