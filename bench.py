@@ -665,6 +665,78 @@ def run_op(args):
             "value": round(work / (med * 1e-3) / scale, 1), "unit": unit, "steps": args.steps}
 
 
+#: plain products of the benchmarked shapes (M, N, K) for the library comparison
+LIBRARY_SHAPES = {
+    "out_2k": (16896, 4608, 4608),
+    "qkv_2k": (16896, 13824, 4608),
+    "up_2k": (16896, 24576, 4608),
+    "down_2k": (16896, 4608, 12288),
+    "qkv_1k": (4608, 13824, 4608),
+    "down_1k": (4608, 4608, 12288),
+    "text_512": (512, 4608, 53248),
+}
+
+
+def run_library_comparison(args):
+    """Our fused linear (zero bias, bf16 out) beside cuBLASLt's NVFP4 GEMM (torch scaled_mm, block-16
+    E4M3 scales plus the fp32 tensor scales) on the same quantised operands: the scale layout of this
+    library is the 32 x 4 x 4 atom layout cuBLASLt reads, so both consume the same bytes.  Prints one
+    JSON line per shape: device times (median of 3 x args.steps back-to-back launches) and the largest
+    difference between the two bf16 outputs."""
+    import torch.nn.functional as F
+    from epilogue_gemm_nvfp4_b200 import binding as B
+    torch.cuda.set_device(0)
+    dev = "cuda"
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        reps = []
+        for _ in range(3):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            for _ in range(args.steps):
+                fn()
+            e.record()
+            torch.cuda.synchronize()
+            reps.append(s.elapsed_time(e) / args.steps)
+        return sorted(reps)[1] * 1e3
+
+    for name, (M, N, K) in LIBRARY_SHAPES.items():
+        gen = torch.Generator(device=dev).manual_seed(1)
+        xq = B.quantize(torch.randn(M, K, device=dev, dtype=torch.bfloat16, generator=gen))
+        wq = B.quantize(torch.randn(N, K, device=dev, dtype=torch.bfloat16, generator=gen) * 0.02)
+        bias = torch.zeros(N, device=dev, dtype=torch.bfloat16)
+        out = torch.empty(M, N, device=dev, dtype=torch.bfloat16)
+        flop = 2.0 * M * N * K
+        res = {"compare": "cublaslt_nvfp4", "shape": name, "M": M, "N": N, "K": K}
+        ours_us = timed(lambda: B.linear(xq, wq, "bias", bias=bias, out=out))
+        B.check_device_error()
+        res.update(ours_us=round(ours_us, 2), ours_tflops=round(flop / ours_us / 1e6, 1))
+        try:
+            sa = [xq.scales.view(torch.float8_e4m3fn), xq.g]
+            sb = [wq.scales.view(torch.float8_e4m3fn), wq.g]
+            recipe = [F.ScalingType.BlockWise1x16, F.ScalingType.TensorWise]
+            swz = [F.SwizzleType.SWIZZLE_32_4_4, F.SwizzleType.NO_SWIZZLE]
+            a4 = xq.codes.view(torch.float4_e2m1fn_x2)
+            b4 = wq.codes.view(torch.float4_e2m1fn_x2).t()
+            lib = lambda: F.scaled_mm(a4, b4, sa, recipe, sb, recipe, swizzle_a=swz, swizzle_b=swz,
+                                      output_dtype=torch.bfloat16)
+            y = lib()
+            res["max_abs_diff"] = float((y.float() - out.float()).abs().max())
+            res["identical"] = bool(torch.equal(y, out))
+            del y
+            lib_us = timed(lib)
+            res.update(cublaslt_us=round(lib_us, 2), cublaslt_tflops=round(flop / lib_us / 1e6, 1),
+                       ours_over_cublaslt=round(lib_us / ours_us, 3))
+        except Exception as e:  # a torch without the NVFP4 path: report, do not fail
+            res["cublaslt"] = f"unavailable: {type(e).__name__}: {str(e)[:200]}"
+        print(json.dumps(res), flush=True)
+        del xq, wq, out
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -674,7 +746,12 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", default=None, help="time one op instead of the block step (profiling / per-config)")
+    ap.add_argument("--compare-cublaslt", action="store_true",
+                    help="time the plain NVFP4 products of the benchmarked shapes beside cuBLASLt's NVFP4 GEMM")
     args = ap.parse_args()
+    if args.compare_cublaslt:
+        run_library_comparison(args)
+        return
     if args.op is not None:
         for name in args.op.split(","):
             args.op = name
