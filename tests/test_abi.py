@@ -40,6 +40,21 @@ def test_scale_helpers_match_the_layout_definition(lib):
         assert lib.nvfp4_scale_offset(r, kb, cols) == O.scale_atom_offset(r, kb, cols)
 
 
+def test_scale_atoms_form_the_rows_the_gemm_tma_reads(lib):
+    """The pair GEMM loads block scales with TMA over the scale bytes viewed as rows of one 512-byte
+    atom: row b * k_atoms + k holds the scales of blocks 4k..4k+3 of rows 128b..128b+127, so the scales
+    of one stage (four K atoms of one 128-row block) are a box of four consecutive rows, and a tensor's
+    scale buffer is a whole number of such rows."""
+    rng = np.random.default_rng(1)
+    for cols in (64, 272, 4608, 12288, 53248):
+        k_atoms = (cols // 16 + 3) // 4
+        for _ in range(300):
+            r, kb = int(rng.integers(0, 1000)), int(rng.integers(0, cols // 16))
+            assert lib.nvfp4_scale_offset(r, kb, cols) // 512 == (r // 128) * k_atoms + kb // 4
+        for rows in (1, 128, 1000):
+            assert lib.nvfp4_scale_bytes(rows, cols) == (rows + 127) // 128 * k_atoms * 512
+
+
 def test_tile_choice_depends_on_n_k_kind_only(lib):
     assert B.tile_n(13824, 4608, "qknorm") == 256
     assert B.tile_n(24576, 4608, "gated_silu") == 256
