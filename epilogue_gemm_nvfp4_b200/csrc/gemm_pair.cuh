@@ -2,7 +2,7 @@
 //
 // A cluster of two CTAs on neighbouring SMs owns a 256 x 256 output tile.  CTA r holds rows
 // [128r, 128r+128) of A and rows [128r, 128r+128) of the tile's 256 B rows in its shared memory.  The
-// leader's (rank 0) single MMA thread issues tcgen05.mma.cta_group::2 with M = 256, N = 256, which
+// leader's (rank 0) MMA warp issues tcgen05.mma.cta_group::2 with M = 256, N = 256, which
 // reads both CTAs' shared memory and writes each CTA's 128 rows of D into that CTA's TMEM.  Each SM
 // therefore receives half of the B codes it would load for a one-CTA 128 x 256 tile: a third less
 // TMA and shared-memory traffic per FLOP, and a stage of 38 KB instead of 54 KB (5 stages).
@@ -15,8 +15,8 @@
 //              Per stage it copies the stage's twelve scale atoms from both CTAs' shared memory into
 //              their TMEM scale slot (tcgen05.cp, which the tensor pipe runs in order with the MMAs
 //              that follow), then issues the four MMAs; commits go to both CTAs' `empty` / `acc_full`.
-//   warp 2     TMEM allocation (paired form).
-//   warps 3-7  idle.
+//   warp 2     TMEM allocation (paired form) before the roles start and release after they end.
+//   warps 2-7  idle while the roles run.
 //   warps 8-15 epilogue of this CTA's 128 rows; the accumulator release is an arrival on the
 //              leader's `acc_empty` (16 arrivals: 8 warps per CTA).
 // 128-wide tiles stay on the one-CTA kernel.  Split-K units exchange partial sums per (pair tile,
